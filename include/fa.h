@@ -1,0 +1,164 @@
+/*
+ * io_aware_exact_32_b200 -- exact IO-aware fused attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Plain pointers and sizes only; no C++ or framework types cross it.
+ *
+ * The operation is exact scaled-dot-product attention,
+ *     O = softmax(scale * Q K^T [+ causal mask]) V,
+ * with Q in R^{Nq x d} and K, V in R^{Nk x d} per (batch, head)
+ * ("Transformer、注意力机制与优化", section 数学公式; the (batch, heads, seq,
+ * head_dim) layout of "优化的注意力实现 (FlashAttention)", section 优势与集成).
+ *
+ * Conventions shared by every call:
+ *  - Tensors are contiguous row-major [B, H, N, d] with d innermost, element
+ *    type bf16 (IEEE bfloat16, 2 bytes), unless stated otherwise.  LSE, D and
+ *    workspaces are fp32.
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates, frees or retains device memory; it keeps one static
+ *    status word per device (see fa_get_device_error).
+ *  - Every tensor pointer must be 16-byte aligned (the TMA engine requires it);
+ *    otherwise FA_ERR_MISALIGNED is returned and nothing is launched.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).  Arguments are validated on the host
+ *    before anything is launched; on any error nothing is launched.
+ *  - Supported head dimensions: d = 64 and d = 128 (FA_ERR_UNSUPPORTED otherwise).
+ *  - causal != 0 applies the lower-triangle mask aligned to the bottom-right
+ *    corner: key j is visible to query i iff j <= i + (Nk - Nq).  For Nq == Nk
+ *    this is tril(diagonal=0).  A query row that sees no key gets O = 0 and
+ *    LSE = -inf.
+ *  - LSE is the natural log of sum_j exp(scale * q_i . k_j) over visible keys.
+ *  - Gradients are overwritten, not accumulated.
+ *  - No exception, abort or exit crosses this boundary.
+ *  - Device-side waits are bounded; a wait that gives up records
+ *    FA_ERR_TIMEOUT in the device status word and the kernel returns.
+ */
+#ifndef IO_AWARE_EXACT_32_B200_FA_H
+#define IO_AWARE_EXACT_32_B200_FA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad scale */
+  FA_ERR_UNSUPPORTED = 2,  /* d not in {64, 128}, or a size beyond the limits below */
+  FA_ERR_MISALIGNED = 3,   /* a tensor pointer not 16-byte aligned */
+  FA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than the *_workspace_size query */
+  FA_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed (launch, tensor map) */
+  FA_ERR_TIMEOUT = 6       /* a bounded device wait gave up (reported by fa_get_device_error) */
+} fa_status;
+
+/*
+ * Forward pass: O and LSE in one fused pass.
+ *
+ * Follows the tiled forward with the online-softmax recurrence (running max m,
+ * running sum l, rescaled output accumulator) of "Transformer、注意力机制与优化",
+ * sections 安全 Softmax 与在线 Softmax and FlashAttention-2 算法, with the
+ * deferred normalisation and the single saved statistic L = m + log(l) of
+ * "FlashAttention 系列技术详解", section 具体优化策略.  The N x N score
+ * matrix never reaches device memory.
+ *
+ *   q    [B, H, Nq, d] bf16, read
+ *   k, v [B, H, Nk, d] bf16, read
+ *   o    [B, H, Nq, d] bf16, written
+ *   lse  [B, H, Nq] fp32, written (natural log; -inf for rows with no visible key)
+ *   scale: multiplies q.k before the softmax (finite, > 0); usually 1/sqrt(d)
+ * Limits: 0 <= B*H <= 2^31-1, 0 <= Nq, Nk <= 2^24.  Nq == 0 or B*H == 0 is a
+ * no-op; Nk == 0 writes O = 0 and LSE = -inf.
+ */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                 void* stream);
+
+/*
+ * Bytes of fp32 workspace fa_bwd needs: D [B, H, Nq] plus the dQ accumulator
+ * [B, H, Nq, d], each region 256-byte aligned.  Returns 0 on invalid sizes.
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int H, int Nq, int d);
+
+/*
+ * Backward pass by recomputation: dQ, dK, dV from Q, K, V, O, dO and the
+ * saved LSE, never storing the N x N matrices.
+ *
+ * Follows "FlashAttention 的基本原理", section 2.4 反向传播 (recompute the
+ * scores and P from the saved statistics; dV = P^T dO, dP = dO V^T, the
+ * row-softmax gradient dS, dQ = dS K, dK = dS^T Q), with D_i = rowsum(dO_i * O_i)
+ * and P recomputed from LSE alone ("FlashAttention 系列技术详解", section
+ * 具体优化策略), and the column-block parallel schedule whose dQ partial sums
+ * meet through atomic adds in device memory ("Transformer、注意力机制与优化",
+ * section 为什么前向传播和反向传播的并行化策略不同).  dQ is therefore not
+ * bitwise deterministic run to run.
+ *
+ *   q, o, dO [B, H, Nq, d] bf16, read;  k, v [B, H, Nk, d] bf16, read
+ *   lse      [B, H, Nq] fp32, read (as written by fa_fwd)
+ *   dq       [B, H, Nq, d] bf16, written;  dk, dv [B, H, Nk, d] bf16, written
+ *   workspace: device fp32 scratch of at least fa_bwd_workspace_size() bytes,
+ *              caller-owned, contents on entry ignored, garbage on exit
+ * Same limits and mask convention as fa_fwd.
+ */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                 const float* lse, void* dq, void* dk, void* dv,
+                 void* workspace, size_t ws_bytes,
+                 int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                 void* stream);
+
+/*
+ * Bytes of workspace fa_decode_splitkv needs for the per-split partial
+ * results (m, l, unnormalised O) at the given split count (0 = the automatic
+ * choice for this Lmax).  Returns 0 on invalid sizes.
+ */
+FA_API size_t fa_decode_workspace_size(int B, int H, int Lmax, int d, int num_splits);
+
+/*
+ * Split-KV decode: one query per (batch, head) against a KV cache with ragged
+ * per-sequence lengths.  The keys of each sequence are cut into chunks that
+ * are processed in parallel; each chunk yields partial (m, l, O~) and a second
+ * kernel merges the partials with the two-block identity for m and l
+ * ("Transformer、注意力机制与优化", sections Flash-Decoding and 安全 Softmax
+ * 与在线 Softmax).  The result does not depend on the split count beyond
+ * rounding.
+ *
+ *   q        [B, H, 1, d] bf16, read
+ *   k_cache, v_cache [B, H, Lmax, d] bf16, read; slots at or beyond
+ *            seqlens[b] are never read
+ *   seqlens  [B] int32 DEVICE array, 1 <= seqlens[b] <= Lmax (values outside
+ *            are clamped to [0, Lmax]; a length of 0 gives O = 0, LSE = -inf)
+ *   o        [B, H, 1, d] bf16, written
+ *   lse      [B, H] fp32, written; may be NULL
+ *   num_splits: chunks per sequence at Lmax (0 = automatic; at most 256)
+ *   workspace: device scratch of at least fa_decode_workspace_size() bytes
+ * Limits: 1 <= Lmax <= 2^24, 0 <= B*H <= 2^31-1.
+ */
+FA_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                            const int* seqlens, int Lmax, void* o, float* lse,
+                            int B, int H, int d, float scale, int num_splits,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the calling device's status
+ * word: FA_OK, or FA_ERR_TIMEOUT if a device-side wait gave up since the last
+ * call.  Returns FA_ERR_CUDA if the synchronisation itself failed.
+ */
+FA_API fa_status fa_get_device_error(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+FA_API const char* fa_status_string(fa_status status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IO_AWARE_EXACT_32_B200_FA_H */

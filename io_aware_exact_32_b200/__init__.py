@@ -1,0 +1,220 @@
+"""io_aware_exact_32_b200: exact IO-aware fused attention for NVIDIA B200 (sm_100a).
+
+The compute lives in a C-ABI shared library (``libfa_sm100.so``, declared in
+``include/fa.h``).  This module only marshals arguments: it checks shapes,
+dtypes and devices, passes raw device pointers and the current CUDA stream,
+and raises on a non-zero status.  PyTorch provides device memory and streams.
+
+C-ABI mirrors (same names, torch tensors in place of pointers):
+    fa_fwd, fa_bwd, fa_bwd_workspace_size, fa_decode_splitkv,
+    fa_decode_workspace_size, fa_get_device_error, fa_status_string, fa_version
+Convenience wrappers that allocate outputs:
+    attention_forward, attention_backward, decode_splitkv
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "FAError", "lib", "lib_path",
+    "fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_decode_splitkv", "fa_decode_workspace_size",
+    "fa_get_device_error", "fa_status_string", "fa_version",
+    "attention_forward", "attention_backward", "decode_splitkv",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libfa_sm100.so")
+
+FA_OK = 0
+_STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_MISALIGNED",
+                 4: "FA_ERR_WORKSPACE", 5: "FA_ERR_CUDA", 6: "FA_ERR_TIMEOUT"}
+
+
+class FAError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {_STATUS_NAMES.get(code, code)} ({fa_status_string(code)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C-ABI library; raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(lib_path):
+        raise ImportError(f"{lib_path} is missing: build it with `python -m io_aware_exact_32_b200.build`")
+    L = ctypes.CDLL(lib_path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    L.fa_fwd.restype = i
+    L.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    L.fa_bwd_workspace_size.restype = sz
+    L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, vp]
+    L.fa_bwd.restype = i
+    L.fa_decode_workspace_size.argtypes = [i, i, i, i, i]
+    L.fa_decode_workspace_size.restype = sz
+    L.fa_decode_splitkv.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, f, i, vp, sz, vp]
+    L.fa_decode_splitkv.restype = i
+    L.fa_get_device_error.argtypes = [vp]
+    L.fa_get_device_error.restype = i
+    L.fa_status_string.argtypes = [i]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_version.argtypes = []
+    L.fa_version.restype = i
+    _lib = L
+    return L
+
+
+def fa_status_string(code: int) -> str:
+    return lib().fa_status_string(int(code)).decode()
+
+
+def fa_version() -> int:
+    return lib().fa_version()
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check(code: int, where: str):
+    if code != FA_OK:
+        raise FAError(code, where)
+
+
+def _need(t, name, dtype, device, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _scale(scale, d):
+    return float(1.0 / math.sqrt(d) if scale is None else scale)
+
+
+# ------------------------------------------------------------------------------ C-ABI mirrors
+def fa_fwd(q, k, v, o, lse, causal: bool, scale=None, stream=None) -> None:
+    """O, LSE of exact attention (see include/fa.h: fa_fwd).  q/o [B,H,Nq,d], k/v [B,H,Nk,d] bf16, lse [B,H,Nq] fp32."""
+    import torch
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k, "k", torch.bfloat16, dev, (B, H, Nk, d))
+    _need(v, "v", torch.bfloat16, dev, (B, H, Nk, d))
+    _need(o, "o", torch.bfloat16, dev, (B, H, Nq, d))
+    _need(lse, "lse", torch.float32, dev, (B, H, Nq))
+    _check(lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                        _scale(scale, d), int(bool(causal)), _stream_ptr(stream)), "fa_fwd")
+
+
+def fa_bwd_workspace_size(B: int, H: int, Nq: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_size(B, H, Nq, d))
+
+
+def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal: bool, scale=None, stream=None) -> None:
+    """dQ, dK, dV by recomputation (see include/fa.h: fa_bwd).  workspace: uint8 device tensor."""
+    import torch
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    dev = q.device
+    for t, n, shp in ((q, "q", (B, H, Nq, d)), (o, "o", (B, H, Nq, d)), (dO, "dO", (B, H, Nq, d)),
+                      (dq, "dq", (B, H, Nq, d)), (k, "k", (B, H, Nk, d)), (v, "v", (B, H, Nk, d)),
+                      (dk, "dk", (B, H, Nk, d)), (dv, "dv", (B, H, Nk, d))):
+        _need(t, n, torch.bfloat16, dev, shp)
+    _need(lse, "lse", torch.float32, dev, (B, H, Nq))
+    _need(workspace, "workspace", torch.uint8, dev)
+    _check(lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                        _ptr(workspace), workspace.numel(), B, H, Nq, Nk, d, _scale(scale, d),
+                        int(bool(causal)), _stream_ptr(stream)), "fa_bwd")
+
+
+def fa_decode_workspace_size(B: int, H: int, Lmax: int, d: int, num_splits: int = 0) -> int:
+    return int(lib().fa_decode_workspace_size(B, H, Lmax, d, num_splits))
+
+
+def fa_decode_splitkv(q, k_cache, v_cache, seqlens, o, lse, workspace, scale=None, num_splits: int = 0,
+                      stream=None) -> None:
+    """Split-KV decode (see include/fa.h: fa_decode_splitkv).  q/o [B,H,1,d], caches [B,H,Lmax,d], seqlens int32 [B]."""
+    import torch
+    B, H, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query per (batch, head)")
+    Lmax = k_cache.shape[2]
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev, (B, H, Lmax, d))
+    _need(v_cache, "v_cache", torch.bfloat16, dev, (B, H, Lmax, d))
+    _need(seqlens, "seqlens", torch.int32, dev, (B,))
+    _need(o, "o", torch.bfloat16, dev, (B, H, 1, d))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev, (B, H))
+    _need(workspace, "workspace", torch.uint8, dev)
+    _check(lib().fa_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(o), _ptr(lse),
+                                   B, H, d, _scale(scale, d), int(num_splits), _ptr(workspace), workspace.numel(),
+                                   _stream_ptr(stream)), "fa_decode_splitkv")
+
+
+def fa_get_device_error(stream=None) -> int:
+    return int(lib().fa_get_device_error(_stream_ptr(stream)))
+
+
+# ------------------------------------------------------------------------------ conveniences
+def _workspace(nbytes: int, device):
+    import torch
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def attention_forward(q, k, v, causal: bool = False, scale=None, stream=None):
+    """Allocate O and LSE and run fa_fwd; returns (o, lse)."""
+    import torch
+    B, H, Nq, d = q.shape
+    o = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    fa_fwd(q, k, v, o, lse, causal, scale, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, dO, causal: bool = False, scale=None, stream=None, workspace=None):
+    """Allocate dQ, dK, dV (and the workspace unless given) and run fa_bwd; returns (dq, dk, dv)."""
+    import torch
+    B, H, Nq, d = q.shape
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    if workspace is None:
+        workspace = _workspace(fa_bwd_workspace_size(B, H, Nq, d), q.device)
+    fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal, scale, stream)
+    return dq, dk, dv
+
+
+def decode_splitkv(q, k_cache, v_cache, seqlens, scale=None, num_splits: int = 0, stream=None, workspace=None):
+    """Allocate O, LSE (and the workspace unless given) and run fa_decode_splitkv; returns (o, lse)."""
+    import torch
+    B, H, _, d = q.shape
+    o = torch.empty((B, H, 1, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = _workspace(fa_decode_workspace_size(B, H, k_cache.shape[2], d, num_splits), q.device)
+    fa_decode_splitkv(q, k_cache, v_cache, seqlens, o, lse, workspace, scale, num_splits, stream)
+    return o, lse

@@ -1,0 +1,406 @@
+// Attention backward for sm_100a by recomputation.
+//
+// Method ("FlashAttention 的基本原理", section 2.4 反向传播; "FlashAttention 系列技术详解",
+// sections 反向传播步骤 and 具体优化策略): the forward saved only O and L = logsumexp.  For
+// every (query block i, key block j) the scores are recomputed, P = exp(scale S - L), and
+//   dV_j += P^T dO_i,  dP = dO_i V_j^T,  dS = P * (dP - D_i),  dK_j += scale dS^T Q_i,
+//   dQ_i += scale dS K_j,  with D_i = rowsum(dO_i * O_i).
+// Work is split over key/value blocks ("Transformer、注意力机制与优化", section 为什么前向
+// 传播和反向传播的并行化策略不同): each CTA owns one key block, keeps dK_j and dV_j on chip, and
+// adds its dQ_i contributions to an fp32 accumulator in device memory with atomic adds.
+//
+// Kernels:
+//   fa_bwd_preprocess_kernel  D = rowsum(dO * O) (fp32) and zero the dQ accumulator
+//   fa_bwd_main_kernel        the loop above for one 128-key block per CTA (tcgen05 + TMA)
+//   fa_bwd_dq_convert_kernel  dQ accumulator (fp32) -> dQ (bf16)
+//
+// Main-kernel layout (computed transposed, keys on TMEM lanes, so that dK/dV rows and the
+// P^T operand of dV = P^T dO live on the lane that owns the key):
+//   TMEM: S^T (128 cols) | dP^T (128 cols; later reused for the dQ block) | dV (d) | dK (d)
+//   SMEM: K_j, V_j (resident), a ring of (Q_i, dO_i) stages, dS^T (bf16, 128-byte swizzle)
+//   warps 0-3: one thread per key row: P, dS, dQ read-out + atomics, dK/dV epilogue
+//   warp 4: tcgen05 MMA issuer; warp 5: TMA producer.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdTraits {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int NBOX = D / 64;
+  static constexpr int BOX_BYTES = 128 * 64 * 2;       // 16 KB
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // 128 x D bf16
+  static constexpr int NS = (D == 64) ? 3 : 2;         // (Q, dO) stages
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = TILE_BYTES;
+  static constexpr int OFF_QD = 2 * TILE_BYTES;              // stage s: Q at +0, dO at +TILE_BYTES
+  static constexpr int OFF_DS = OFF_QD + NS * 2 * TILE_BYTES;  // 128 keys x 128 queries bf16 = 32 KB
+  static constexpr int OFF_STAT = OFF_DS + 2 * BOX_BYTES;      // [2][128] fp32: LSE*log2e, D
+  static constexpr int OFF_BAR = OFF_STAT + 2 * 128 * 4;
+  // barriers: kv_full | qd_full[NS] | qd_empty[NS] | s_full | ds_ready | dq_full | dq_free | acc_done | drain
+  static constexpr int BAR_KV = 0;
+  static constexpr int BAR_QD_FULL = 1;
+  static constexpr int BAR_QD_EMPTY = 1 + NS;
+  static constexpr int BAR_S_FULL = 1 + 2 * NS;
+  static constexpr int BAR_DS_READY = BAR_S_FULL + 1;
+  static constexpr int BAR_DQ_FULL = BAR_S_FULL + 2;
+  static constexpr int BAR_DQ_FREE = BAR_S_FULL + 3;
+  static constexpr int BAR_ACC_DONE = BAR_S_FULL + 4;
+  static constexpr int BAR_DRAIN = BAR_S_FULL + 5;
+  static constexpr int NBAR = BAR_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t IDESC_SQ = make_idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
+  static constexpr uint32_t IDESC_DVK = make_idesc_bf16(128, D, false, true);    // P^T dO, dS^T Q
+  static constexpr uint32_t IDESC_DQ = make_idesc_bf16(128, D, true, true);      // dS K
+};
+
+struct BwdParams {
+  const float* lse;   // [BH, Nq]
+  const float* dvec;  // [BH, Nq]
+  float* dq_acc;      // [BH, Nq, D]
+  __nv_bfloat16* dk;  // [BH, Nk, D]
+  __nv_bfloat16* dv;  // [BH, Nk, D]
+  int Nq, Nk, BH, nkt;
+  float scale, scale_log2;
+  int causal;
+};
+
+// ---------------------------------------------------------------------------------------------
+// D_i = sum_k dO_ik O_ik and dQ accumulator zeroing.  One warp per query row.
+// ---------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
+                                                                const __nv_bfloat16* __restrict__ dout,
+                                                                float* __restrict__ dvec,
+                                                                float* __restrict__ dq_acc, long long rows) {
+  const long long row = blockIdx.x * 8ll + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  constexpr int PER = D / 32;  // elements per lane (2 or 4)
+  const __nv_bfloat16* orow = o + row * D + lane * PER;
+  const __nv_bfloat16* drow = dout + row * D + lane * PER;
+  float acc = 0.f;
+  if constexpr (PER == 4) {
+    const uint2 a = *reinterpret_cast<const uint2*>(orow);
+    const uint2 b = *reinterpret_cast<const uint2*>(drow);
+    acc = bf16lo_to_f32(a.x) * bf16lo_to_f32(b.x) + bf16hi_to_f32(a.x) * bf16hi_to_f32(b.x) +
+          bf16lo_to_f32(a.y) * bf16lo_to_f32(b.y) + bf16hi_to_f32(a.y) * bf16hi_to_f32(b.y);
+  } else {
+    const uint32_t a = *reinterpret_cast<const uint32_t*>(orow);
+    const uint32_t b = *reinterpret_cast<const uint32_t*>(drow);
+    acc = bf16lo_to_f32(a) * bf16lo_to_f32(b) + bf16hi_to_f32(a) * bf16hi_to_f32(b);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) dvec[row] = acc;
+  float* qrow = dq_acc + row * D + lane * PER;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) qrow[i] = 0.f;
+}
+
+// dQ accumulator (already scaled) -> bf16, 8 elements per thread.
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ acc,
+                                                                __nv_bfloat16* __restrict__ dq, long long n8) {
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  reinterpret_cast<uint4*>(dq)[i] =
+      make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+}
+
+// First query block that sees key k0, under the bottom-right causal alignment.
+__device__ __forceinline__ int bwd_first_q_tile(int k0, int Nq, int Nk, int causal) {
+  if (!causal) return 0;
+  const int qmin = k0 - (Nk - Nq);
+  return qmin <= 0 ? 0 : qmin / 128;
+}
+
+template <int D>
+__device__ __forceinline__ void bwd_issue_ss_kmajor(uint32_t tmem_d, uint32_t a_smem, uint32_t b_smem) {
+  using T = BwdTraits<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * T::BOX_BYTES + (kk % 4) * 32;
+    mma_ss(tmem_d, make_sdesc_sw128(a_smem + off, 16, 1024), make_sdesc_sw128(b_smem + off, 16, 1024),
+           T::IDESC_SQ, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                       const BwdParams p) {
+  using T = BwdTraits<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + T::OFF_BAR + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::OFF_MISC + 4);
+  float* stat = reinterpret_cast<float*>(smem + T::OFF_STAT);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % p.BH;
+  const int jt = blockIdx.x / p.BH;
+  const int k0 = jt * 128;
+  const int nqt = (p.Nq + 127) / 128;
+  const int i0 = bwd_first_q_tile(k0, p.Nq, p.Nk, p.causal);
+  const int n_q = max(0, nqt - i0);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(T::BAR_KV), 1);
+    for (int s = 0; s < T::NS; ++s) {
+      mbar_init(bar(T::BAR_QD_FULL + s), 1);
+      mbar_init(bar(T::BAR_QD_EMPTY + s), 1);
+    }
+    mbar_init(bar(T::BAR_S_FULL), 1);
+    mbar_init(bar(T::BAR_DS_READY), 128);
+    mbar_init(bar(T::BAR_DQ_FULL), 1);
+    mbar_init(bar(T::BAR_DQ_FREE), 128);
+    mbar_init(bar(T::BAR_ACC_DONE), 1);
+    mbar_init(bar(T::BAR_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 5 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmDO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------------ compute warpgroup
+    const int r = warp * 32 + lane;  // key row in the block == TMEM lane; also the dQ query row
+    const int key = k0 + r;
+    const bool key_ok = key < p.Nk;
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(warp * 32) << 16);
+    // Query column c of block i sees this key iff c >= cmin (bottom-right causal alignment).
+    const int shift = key - (p.Nk - p.Nq);
+    const uint32_t ds_row = sbase + T::OFF_DS + r * 128;
+    bool ok = true;
+    for (int it = 0; it < n_q; ++it) {
+      const int q0 = (i0 + it) * 128;
+      // Per-block statistics: LSE in log2 units (+inf past Nq) and D.  The first barrier keeps
+      // the previous block's readers ahead of the overwrite, the second publishes the new values.
+      float* st = stat;
+      {
+        const int q = q0 + r;
+        const bool in = q < p.Nq;
+        const size_t gi = (size_t)bh * p.Nq + (in ? q : 0);
+        const float lse2 = in ? p.lse[gi] * kLog2e : INFINITY;
+        const float dd = in ? p.dvec[gi] : 0.f;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        st[r] = lse2;
+        st[128 + r] = dd;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL), it & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int cmin = p.causal ? shift - q0 : -1;
+#pragma unroll 1
+      for (int c32 = 0; c32 < 4; ++c32) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld32x32b_x32_wait(lane_addr + T::COL_S + 32 * c32, sv);
+        tmem_ld32x32b_x32_wait(lane_addr + T::COL_DP + 32 * c32, dpv);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const int c = 32 * c32 + i;
+          const bool v0 = key_ok && (c >= cmin), v1 = key_ok && (c + 1 >= cmin);
+          const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sv[i]), p.scale_log2, -st[c])) : 0.f;
+          const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sv[i + 1]), p.scale_log2, -st[c + 1])) : 0.f;
+          const float d0 = p0 * (__uint_as_float(dpv[i]) - st[128 + c]);
+          const float d1 = p1 * (__uint_as_float(dpv[i + 1]) - st[128 + c + 1]);
+          pk[i / 2] = pack_bf16x2(p0, p1);
+          dk[i / 2] = pack_bf16x2(d0, d1);
+        }
+        // P^T chunk -> TMEM (first 64 columns of the S^T block, bf16 pairs).
+        tmem_st32x32b_x16(lane_addr + T::COL_S + 16 * c32, pk);
+        // dS^T chunk -> shared memory, K-major with 128-byte swizzle (box = 64 query columns).
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int kc = 4 * c32 + m;  // 16-byte chunk index along the 128 query columns
+          const uint32_t addr = ds_row + (kc >> 3) * T::BOX_BYTES + (((kc & 7) ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk[4 * m]), "r"(dk[4 * m + 1]),
+                       "r"(dk[4 * m + 2]), "r"(dk[4 * m + 3])
+                       : "memory");
+        }
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(T::BAR_DS_READY));
+      // dQ block (query rows on lanes) -> scale -> atomic add into the fp32 accumulator.
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DQ_FULL), it & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const int q = q0 + r;
+        float* dst = p.dq_acc + ((size_t)bh * p.Nq + (q < p.Nq ? q : 0)) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32x32b_x32_wait(lane_addr + T::COL_DP + 32 * c, v);
+          if (q < p.Nq) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float4 a = make_float4(__uint_as_float(v[4 * i]) * p.scale, __uint_as_float(v[4 * i + 1]) * p.scale,
+                                     __uint_as_float(v[4 * i + 2]) * p.scale, __uint_as_float(v[4 * i + 3]) * p.scale);
+              atomicAdd(reinterpret_cast<float4*>(dst + 32 * c + 4 * i), a);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(T::BAR_DQ_FREE));
+    }
+    // dK, dV epilogue.
+    if (ok && n_q > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_ACC_DONE), 0, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      const size_t off = ((size_t)bh * p.Nk + (key_ok ? key : 0)) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* out = (which ? p.dk : p.dv) + off;
+        const float mul = which ? p.scale : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (n_q > 0) {
+            tmem_ld32x32b_x32_wait(lane_addr + (which ? T::COL_DK : T::COL_DV) + 32 * c, v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
+          if (key_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]) * mul, __uint_as_float(v[8 * i + 1]) * mul),
+                                  pack_bf16x2(__uint_as_float(v[8 * i + 2]) * mul, __uint_as_float(v[8 * i + 3]) * mul),
+                                  pack_bf16x2(__uint_as_float(v[8 * i + 4]) * mul, __uint_as_float(v[8 * i + 5]) * mul),
+                                  pack_bf16x2(__uint_as_float(v[8 * i + 6]) * mul, __uint_as_float(v[8 * i + 7]) * mul));
+          }
+        }
+      }
+    } else {
+      *abort_flag = 1;
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_q > 0) {
+      const uint32_t k_smem = sbase + T::OFF_K, v_smem = sbase + T::OFF_V, ds_smem = sbase + T::OFF_DS;
+      const uint32_t tS = tmem_base + T::COL_S, tDP = tmem_base + T::COL_DP;
+      const uint32_t tDV = tmem_base + T::COL_DV, tDK = tmem_base + T::COL_DK;
+      auto q_smem = [&](int it) { return sbase + T::OFF_QD + (it % T::NS) * 2 * T::TILE_BYTES; };
+      bool ok = mbar_wait(bar(T::BAR_KV), 0, abort_flag);
+      if (ok) ok = mbar_wait(bar(T::BAR_QD_FULL + 0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(0));                  // S^T = K Q^T
+        bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(0) + T::TILE_BYTES);  // dP^T = V dO^T
+        mma_commit(bar(T::BAR_S_FULL));
+      }
+      for (int it = 0; ok && it < n_q; ++it) {
+        const uint32_t qs = q_smem(it), dos = qs + T::TILE_BYTES;
+        if (!(ok = mbar_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
+        tc_fence_after();
+        // dQ_i = dS K_j -> dP^T columns (dP^T is already consumed).  A = dS (MN-major view of dS^T).
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tDP, make_sdesc_sw128(ds_smem + kk * 2048, T::BOX_BYTES, 1024),
+                 make_sdesc_sw128(k_smem + kk * 2048, T::BOX_BYTES, 1024), T::IDESC_DQ, kk > 0 ? 1u : 0u);
+        mma_commit(bar(T::BAR_DQ_FULL));
+        // dV_j += P^T dO_i  (P^T from TMEM, dO MN-major).
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tDV, tS + kk * 8, make_sdesc_sw128(dos + kk * 2048, T::BOX_BYTES, 1024), T::IDESC_DVK,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        // dK_j += dS^T Q_i  (dS^T K-major, Q MN-major); scale is applied in the epilogue.
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tDK, make_sdesc_sw128(ds_smem + (kk / 4) * T::BOX_BYTES + (kk % 4) * 32, 16, 1024),
+                 make_sdesc_sw128(qs + kk * 2048, T::BOX_BYTES, 1024), T::IDESC_DVK, (it > 0 || kk > 0) ? 1u : 0u);
+        if (it + T::NS < n_q) mma_commit(bar(T::BAR_QD_EMPTY + it % T::NS));
+        if (it + 1 < n_q) {
+          const uint32_t qn = q_smem(it + 1);
+          if (!(ok = mbar_wait(bar(T::BAR_QD_FULL + (it + 1) % T::NS), ((it + 1) / T::NS) & 1, abort_flag))) break;
+          tc_fence_after();
+          bwd_issue_ss_kmajor<D>(tS, k_smem, qn);  // after dV in issue order: P^T already read
+          if (!(ok = mbar_wait(bar(T::BAR_DQ_FREE), it & 1, abort_flag))) break;
+          tc_fence_after();
+          bwd_issue_ss_kmajor<D>(tDP, v_smem, qn + T::TILE_BYTES);
+          mma_commit(bar(T::BAR_S_FULL));
+        }
+      }
+      if (ok) mma_commit(bar(T::BAR_ACC_DONE));
+      if (!ok) {
+        *abort_flag = 1;
+        mma_commit(bar(T::BAR_DRAIN));
+        const volatile int never = 0;
+        mbar_wait(bar(T::BAR_DRAIN), 0, &never);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_q > 0) {
+      mbar_arrive_expect_tx(bar(T::BAR_KV), 2 * T::TILE_BYTES);
+      for (int b = 0; b < T::NBOX; ++b) {
+        tma_load_3d(sbase + T::OFF_K + b * T::BOX_BYTES, &tmK, bar(T::BAR_KV), 64 * b, k0, bh);
+        tma_load_3d(sbase + T::OFF_V + b * T::BOX_BYTES, &tmV, bar(T::BAR_KV), 64 * b, k0, bh);
+      }
+      bool ok = true;
+      int issued = 0;
+      for (int it = 0; it < n_q; ++it) {
+        const int s = it % T::NS;
+        if (!(ok = mbar_wait(bar(T::BAR_QD_EMPTY + s), ((it / T::NS) & 1) ^ 1, abort_flag))) break;
+        mbar_arrive_expect_tx(bar(T::BAR_QD_FULL + s), 2 * T::TILE_BYTES);
+        const uint32_t dst = sbase + T::OFF_QD + s * 2 * T::TILE_BYTES;
+        const int q0 = (i0 + it) * 128;
+        for (int b = 0; b < T::NBOX; ++b) {
+          tma_load_3d(dst + b * T::BOX_BYTES, &tmQ, bar(T::BAR_QD_FULL + s), 64 * b, q0, bh);
+          tma_load_3d(dst + T::TILE_BYTES + b * T::BOX_BYTES, &tmDO, bar(T::BAR_QD_FULL + s), 64 * b, q0, bh);
+        }
+        issued = it + 1;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        const volatile int never = 0;
+        for (int it = max(0, issued - T::NS); it < issued; ++it)
+          mbar_wait(bar(T::BAR_QD_FULL + it % T::NS), (it / T::NS) & 1, &never);
+        mbar_wait(bar(T::BAR_KV), 0, &never);
+      }
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, T::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,298 @@
+// C-ABI entry points (declared in include/fa.h): argument validation, TMA tensor-map encoding
+// and kernel launches on the caller's stream.  Nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "bwd_sm100.cuh"
+#include "decode_sm100.cuh"
+#include "fwd_sm100.cuh"
+
+namespace {
+
+constexpr int kMaxSeq = 1 << 24;
+constexpr int kMaxSplits = 256;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [BH, N, D] bf16 viewed as a 3-D tensor {D, N, BH}; box = 64 columns x 128 rows x 1, 128-byte swizzle.
+// Rows past N read as zero.
+bool make_map_3d(CUtensorMap* map, const void* base, int D, int N, long long BH) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Opt a kernel into its dynamic shared memory once per device.
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  static std::mutex mu;
+  static const void* done[64][16];
+  static int ndone[64];
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return false;
+  for (int i = 0; i < ndone[dev]; ++i)
+    if (done[dev][i] == reinterpret_cast<const void*>(kernel)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  if (ndone[dev] < 16) done[dev][ndone[dev]++] = reinterpret_cast<const void*>(kernel);
+  return true;
+}
+
+fa_status check_common(int B, int H, int Nq, int Nk, int d, float scale) {
+  if (B < 0 || H < 0 || Nq < 0 || Nk < 0) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Nq > kMaxSeq || Nk > kMaxSeq) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * H > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+int decode_splits(int Lmax, int num_splits) {
+  if (num_splits > 0) return num_splits < kMaxSplits ? num_splits : kMaxSplits;
+  int s = (Lmax + 1023) / 1024;  // about 1024 keys (512 KB of K+V at d = 128) per chunk
+  return s < 1 ? 1 : (s > kMaxSplits ? kMaxSplits : s);
+}
+
+int decode_chunk(int Lmax, int S) {
+  int c = (Lmax + S - 1) / S;
+  return (c + 31) & ~31;
+}
+
+template <int D>
+fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int Nq, int Nk,
+                     float scale, int causal, cudaStream_t stream) {
+  using T = fa::FwdTraits<D>;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_3d(&mq, q, D, Nq, BH) || !make_map_3d(&mk, k, D, Nk, BH) || !make_map_3d(&mv, v, D, Nk, BH))
+    return FA_ERR_CUDA;
+  if (!set_smem(fa::fa_fwd_kernel<D>, T::SMEM_BYTES)) return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.BH = BH;
+  p.npairs = (Nq + 255) / 256;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  const long long blocks = (long long)p.npairs * BH;
+  if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  fa::fa_fwd_kernel<D><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                     void* dq, void* dk, void* dv, void* ws, int BH, int Nq, int Nk, float scale, int causal,
+                     cudaStream_t stream) {
+  using T = fa::BwdTraits<D>;
+  const long long rows = (long long)BH * Nq;
+  float* dvec = static_cast<float*>(ws);
+  float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)rows * 4));
+  if (rows > 0) {
+    fa::fa_bwd_preprocess_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), dvec, dq_acc, rows);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (Nk > 0) {
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_map_3d(&mq, q, D, Nq, BH) || !make_map_3d(&mk, k, D, Nk, BH) || !make_map_3d(&mv, v, D, Nk, BH) ||
+        !make_map_3d(&mdo, dO, D, Nq, BH))
+      return FA_ERR_CUDA;
+    if (!set_smem(fa::fa_bwd_main_kernel<D>, T::SMEM_BYTES)) return FA_ERR_CUDA;
+    fa::BwdParams p;
+    p.lse = lse;
+    p.dvec = dvec;
+    p.dq_acc = dq_acc;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.BH = BH;
+    p.nkt = (Nk + 127) / 128;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    const long long blocks = (long long)p.nkt * BH;
+    if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    fa::fa_bwd_main_kernel<D><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (rows > 0) {
+    const long long n8 = rows * D / 8;
+    fa::fa_bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, stream>>>(
+        dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+template <int D>
+fa_status launch_decode(const void* q, const void* kc, const void* vc, const int* seqlens, int Lmax, void* o,
+                        float* lse, int BH, int H, float scale, int S, void* ws, cudaStream_t stream) {
+  using T = fa::DecTraits<D>;
+  if (!set_smem(fa::fa_decode_split_kernel<D>, T::SMEM_BYTES)) return FA_ERR_CUDA;
+  fa::DecParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<const __nv_bfloat16*>(kc);
+  p.vc = static_cast<const __nv_bfloat16*>(vc);
+  p.seqlens = seqlens;
+  p.part_o = static_cast<float*>(ws);
+  p.part_ml = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)BH * S * D * 4));
+  p.Lmax = Lmax;
+  p.H = H;
+  p.S = S;
+  p.C = decode_chunk(Lmax, S);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long units = (long long)BH * S;
+  if (units > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  fa::fa_decode_split_kernel<D><<<(unsigned)units, T::THREADS, T::SMEM_BYTES, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  fa::fa_decode_merge_kernel<D><<<(unsigned)((BH + 3) / 4), 128, 0, stream>>>(
+      p.part_o, p.part_ml, static_cast<__nv_bfloat16*>(o), lse, BH, S);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                 int d, float scale, int causal, void* stream) {
+  fa_status st = check_common(B, H, Nq, Nk, d, scale);
+  if (st != FA_OK) return st;
+  const long long BH = (long long)B * H;
+  if (BH == 0 || Nq == 0) return FA_OK;
+  if (!q || !o || !lse || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || (Nk > 0 && (!aligned16(k) || !aligned16(v))))
+    return FA_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (Nk == 0) {
+    const long long rows = BH * Nq;
+    const long long n = rows * d;
+    fa::fa_fwd_empty_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(static_cast<__nv_bfloat16*>(o), lse, rows,
+                                                                         d);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  }
+  return d == 64 ? launch_fwd<64>(q, k, v, o, lse, (int)BH, Nq, Nk, scale, causal, s)
+                 : launch_fwd<128>(q, k, v, o, lse, (int)BH, Nq, Nk, scale, causal, s);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int Nq, int d) {
+  if (B < 0 || H < 0 || Nq < 0 || (d != 64 && d != 128)) return 0;
+  const size_t rows = (size_t)B * H * Nq;
+  return align256(rows * 4) + align256(rows * d * 4);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int Nq, int Nk, int d,
+                 float scale, int causal, void* stream) {
+  fa_status st = check_common(B, H, Nq, Nk, d, scale);
+  if (st != FA_OK) return st;
+  const long long BH = (long long)B * H;
+  if (BH == 0 || (Nq == 0 && Nk == 0)) return FA_OK;
+  const bool has_q = Nq > 0, has_k = Nk > 0;
+  if ((has_q && (!q || !o || !dO || !lse || !dq)) || (has_k && (!k || !v || !dk || !dv)))
+    return FA_ERR_INVALID_ARG;
+  if ((has_q && (!aligned16(q) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) || !aligned16(dq))) ||
+      (has_k && (!aligned16(k) || !aligned16(v) || !aligned16(dk) || !aligned16(dv))))
+    return FA_ERR_MISALIGNED;
+  const size_t need = fa_bwd_workspace_size(B, H, Nq, d);
+  if (need > 0 && (!workspace || ws_bytes < need)) return FA_ERR_WORKSPACE;
+  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s)
+                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s);
+}
+
+size_t fa_decode_workspace_size(int B, int H, int Lmax, int d, int num_splits) {
+  if (B < 0 || H < 0 || Lmax < 1 || Lmax > kMaxSeq || (d != 64 && d != 128) || num_splits < 0) return 0;
+  const int S = decode_splits(Lmax, num_splits);
+  const size_t units = (size_t)B * H * S;
+  return align256(units * d * 4) + align256(units * 2 * 4);
+}
+
+fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, int Lmax,
+                            void* o, float* lse, int B, int H, int d, float scale, int num_splits, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  if (B < 0 || H < 0 || num_splits < 0) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Lmax < 1 || Lmax > kMaxSeq) return Lmax < 1 ? FA_ERR_INVALID_ARG : FA_ERR_UNSUPPORTED;
+  if (num_splits > kMaxSplits) return FA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  if (BH == 0) return FA_OK;
+  if (!q || !k_cache || !v_cache || !seqlens || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (lse && !aligned16(lse)) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return FA_ERR_MISALIGNED;
+  const size_t need = fa_decode_workspace_size(B, H, Lmax, d, num_splits);
+  if (!workspace || ws_bytes < need) return FA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_MISALIGNED;
+  const int S = decode_splits(Lmax, num_splits);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode<64>(q, k_cache, v_cache, seqlens, Lmax, o, lse, (int)BH, H, scale, S, workspace, s)
+                 : launch_decode<128>(q, k_cache, v_cache, seqlens, Lmax, o, lse, (int)BH, H, scale, S, workspace, s);
+}
+
+fa_status fa_get_device_error(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return v == 0 ? FA_OK : static_cast<fa_status>(v);
+}
+
+const char* fa_status_string(fa_status status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported size or head dimension";
+    case FA_ERR_MISALIGNED: return "pointer not 16-byte aligned (workspace: 256-byte)";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case FA_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+  }
+  return "unknown status";
+}
+
+int fa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,346 @@
+// Fused attention forward for sm_100a: O = softmax(scale Q K^T [+ causal mask]) V and LSE.
+//
+// Method: the tiled forward of "Transformer、注意力机制与优化" (section FlashAttention-2 算法):
+// a block of query rows stays on chip while key/value blocks stream past it; each row keeps
+// a running max m and running sum l (section 安全 Softmax 与在线 Softmax, two-block identity)
+// and a running output accumulator that is rescaled when m grows ("FlashAttention 的基本原理",
+// section 2.3 前向传播).  Normalisation by l is deferred to the end and only
+// L = m + log(l) is saved for the backward pass ("FlashAttention 系列技术详解", section
+// 具体优化策略).  The score matrix exists only in tensor memory, one 128 x 128 tile at a time.
+//
+// B200 design (not the pages' A100/H100 kernels):
+//  * one CTA owns two 128-row query tiles (Q0, Q1) of one (batch, head) and streams 128-key
+//    K and V tiles through a shared-memory ring filled by TMA (128-byte swizzle);
+//  * one thread issues tcgen05 MMAs: S_t = Q_t K^T (both operands in shared memory) and
+//    O_t += P_t V (P_t read from tensor memory, V from shared memory), fp32 accumulators in
+//    TMEM: S0 | S1 | O0 | O1 = 128 + 128 + d + d columns;
+//  * two softmax warpgroups, one per query tile, each thread owning one row (= one TMEM
+//    lane): while one group exponentiates its S tile, the tensor core runs the other tile's
+//    MMAs (issue order S0 S1 PV0 S0' PV1 S1' PV0' ...);
+//  * exp2 with scale*log2(e) folded into one FMA; the running max is only moved (and O and l
+//    rescaled) when a row's max grows by more than 2^8, which keeps P <= 256 and is exact
+//    because O, l and LSE all use the same stale max;
+//  * P is rounded to bf16 and written over the first half of its own S columns.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdTraits {
+  static_assert(D == 64 || D == 128, "head dim");
+  static constexpr int BM = 128;                       // query rows per tile
+  static constexpr int BN = 128;                       // keys per tile
+  static constexpr int NBOX = D / 64;                  // 64-column TMA boxes per tile
+  static constexpr int BOX_BYTES = 128 * 64 * 2;       // 16 KB
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128 x D bf16 tile
+  static constexpr int NS = (D == 64) ? 6 : 3;         // K/V ring stages
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_KV = 2 * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
+  // barriers: q_full | kv_full[NS] | kv_empty[NS] | s_full[2] | p_ready[2] | o_done[2] | drain
+  static constexpr int BAR_Q = 0;
+  static constexpr int BAR_KV_FULL = 1;
+  static constexpr int BAR_KV_EMPTY = 1 + NS;
+  static constexpr int BAR_S_FULL = 1 + 2 * NS;
+  static constexpr int BAR_P_READY = BAR_S_FULL + 2;
+  static constexpr int BAR_O_DONE = BAR_P_READY + 2;
+  static constexpr int BAR_DRAIN = BAR_O_DONE + 2;
+  static constexpr int NBAR = BAR_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+  static constexpr uint32_t TMEM_COLS = 512;
+  // TMEM columns: S_t at 128 t, O_t at 256 + D t.
+  static __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }
+  static __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + (uint32_t)D * t; }
+  static constexpr int THREADS = 320;  // warps 0-7 softmax, 8 MMA, 9 TMA
+  static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, false, false);
+  static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, false, true);
+};
+
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int Nq, Nk, BH;
+  int npairs;        // ceil(Nq / 256)
+  float scale_log2;  // scale * log2(e)
+  int causal;
+};
+
+// Number of 128-key tiles the CTA owning query rows [q0, q0 + 256) must visit.
+__device__ __forceinline__ int fwd_num_kv_tiles(int q0, int Nq, int Nk, int causal) {
+  const int nkt = (Nk + 127) / 128;
+  if (!causal) return nkt;
+  const int last = min(q0 + 255, Nq - 1);
+  const int kmax = last + Nk - Nq;  // last visible key of the last row
+  if (kmax < 0) return 1;           // every row fully masked: one tile, all -inf
+  return min(nkt, kmax / 128 + 1);
+}
+
+template <int D>
+__device__ __forceinline__ void fwd_issue_qk(uint32_t tmem_d, uint32_t q_smem, uint32_t k_smem) {
+  using T = FwdTraits<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * T::BOX_BYTES + (kk % 4) * 32;
+    mma_ss(tmem_d, make_sdesc_sw128(q_smem + off, 16, 1024), make_sdesc_sw128(k_smem + off, 16, 1024),
+           T::IDESC_QK, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
+  using T = FwdTraits<D>;
+#pragma unroll
+  for (int kk = 0; kk < 128 / 16; ++kk) {
+    // 16 keys per step: P columns advance by 8 (two bf16 per 32-bit column), V rows by 16 x 128 B.
+    mma_ts(tmem_d, tmem_p + kk * 8, make_sdesc_sw128(v_smem + kk * 2048, T::BOX_BYTES, 1024), T::IDESC_PV,
+           (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using T = FwdTraits<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](int i) -> uint32_t { return sbase + T::OFF_BAR + 8 * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x % p.BH;
+  const int rank = blockIdx.x / p.BH;
+  const int pair = p.causal ? (p.npairs - 1 - rank) : rank;  // causal: heaviest tiles first
+  const int q0 = pair * 256;
+  const int n_kv = fwd_num_kv_tiles(q0, p.Nq, p.Nk, p.causal);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(T::BAR_Q), 1);
+    for (int s = 0; s < T::NS; ++s) {
+      mbar_init(bar(T::BAR_KV_FULL + s), 1);
+      mbar_init(bar(T::BAR_KV_EMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(T::BAR_S_FULL + t), 1);
+      mbar_init(bar(T::BAR_P_READY + t), 128);
+      mbar_init(bar(T::BAR_O_DONE + t), 1);
+    }
+    mbar_init(bar(T::BAR_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp < 8) {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // row in the tile == TMEM lane
+    const int row = q0 + 128 * t + r;   // query index within the head
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t colS = T::col_s(t), colO = T::col_o(t);
+    int kmax = p.Nk - 1;  // last visible key of this row (inclusive)
+    if (p.causal) kmax = min(kmax, row + p.Nk - p.Nq);
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL + t), j & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32x32b_x128_wait(lane_addr + colS, sr);
+      float* s = reinterpret_cast<float*>(sr);
+      const int lim = kmax - 128 * j;  // keys [0, lim] of this tile are visible
+      if (__any_sync(0xffffffffu, lim < 127)) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c > lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      const float m_tile = mx * p.scale_log2;
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_tile > m_run + kRescaleThreshold) {
+        alpha = ex2_approx(m_run - m_tile);
+        resc = (j > 0) && (m_run != -INFINITY);
+        m_run = m_tile;
+      }
+      const float base = (m_run == -INFINITY) ? 0.f : m_run;
+      float sum0 = 0.f, sum1 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float e0 = ex2_approx(fmaf(s[2 * c], p.scale_log2, -base));
+        const float e1 = ex2_approx(fmaf(s[2 * c + 1], p.scale_log2, -base));
+        sum0 += e0;
+        sum1 += e1;
+        pk[c] = pack_bf16x2(e0, e1);
+      }
+      l_run = l_run * alpha + (sum0 + sum1);
+      tmem_st32x32b_x64(lane_addr + colS, pk);
+      if (__any_sync(0xffffffffu, resc)) {
+        // O_t still holds the sum through tile j-1: wait until PV(j-1) has landed, then scale.
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (j - 1) & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32x32b_x32_wait(lane_addr + colO + 32 * c, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32x32b_x32(lane_addr + colO + 32 * c, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(T::BAR_P_READY + t));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (n_kv - 1) & 1, abort_flag));
+    if (ok) {
+      tc_fence_after();
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const bool in_range = row < p.Nq;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32x32b_x32_wait(lane_addr + colO + 32 * c, o);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+        if (in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (in_range) p.lse[(size_t)bh * p.Nq + row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+    } else {
+      *abort_flag = 1;
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const int total_loads = 2 * n_kv;
+      auto release = [&](int load_idx) {
+        // Only stages the producer will refill get an "empty" arrival.
+        if (load_idx + T::NS < total_loads) mma_commit(bar(T::BAR_KV_EMPTY + load_idx % T::NS));
+      };
+      const uint32_t q_smem[2] = {sbase + T::OFF_Q, sbase + T::OFF_Q + T::TILE_BYTES};
+      const uint32_t tS[2] = {tmem_base + T::col_s(0), tmem_base + T::col_s(1)};
+      const uint32_t tO[2] = {tmem_base + T::col_o(0), tmem_base + T::col_o(1)};
+      bool ok = mbar_wait(bar(T::BAR_Q), 0, abort_flag);
+      int v_prev = -1;
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int ik = 2 * j, iv = 2 * j + 1;
+        const int sk = ik % T::NS, sv = iv % T::NS;
+        const uint32_t k_smem = sbase + T::OFF_KV + sk * T::TILE_BYTES;
+        const uint32_t v_smem = sbase + T::OFF_KV + sv * T::TILE_BYTES;
+        if (!(ok = mbar_wait(bar(T::BAR_KV_FULL + sk), (ik / T::NS) & 1, abort_flag))) break;
+        tc_fence_after();
+        fwd_issue_qk<D>(tS[0], q_smem[0], k_smem);
+        mma_commit(bar(T::BAR_S_FULL + 0));
+        if (j > 0) {
+          if (!(ok = mbar_wait(bar(T::BAR_P_READY + 1), (j - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, j - 1 > 0);
+          mma_commit(bar(T::BAR_O_DONE + 1));
+          release(v_prev);
+        }
+        fwd_issue_qk<D>(tS[1], q_smem[1], k_smem);
+        mma_commit(bar(T::BAR_S_FULL + 1));
+        release(ik);
+        if (!(ok = mbar_wait(bar(T::BAR_KV_FULL + sv), (iv / T::NS) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(bar(T::BAR_P_READY + 0), j & 1, abort_flag))) break;
+        tc_fence_after();
+        fwd_issue_pv<D>(tO[0], tS[0], v_smem, j > 0);
+        mma_commit(bar(T::BAR_O_DONE + 0));
+        v_prev = iv;
+      }
+      if (ok && (ok = mbar_wait(bar(T::BAR_P_READY + 1), (n_kv - 1) & 1, abort_flag))) {
+        tc_fence_after();
+        fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, n_kv - 1 > 0);
+        mma_commit(bar(T::BAR_O_DONE + 1));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // Let every MMA already issued finish before the CTA releases its tensor memory.
+        mma_commit(bar(T::BAR_DRAIN));
+        const volatile int never = 0;
+        mbar_wait(bar(T::BAR_DRAIN), 0, &never);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(T::BAR_Q), 2 * T::TILE_BYTES);
+      for (int t = 0; t < 2; ++t)
+        for (int b = 0; b < T::NBOX; ++b)
+          tma_load_3d(sbase + T::OFF_Q + t * T::TILE_BYTES + b * T::BOX_BYTES, &tmQ, bar(T::BAR_Q), 64 * b,
+                      q0 + 128 * t, bh);
+      const int total_loads = 2 * n_kv;
+      bool ok = true;
+      int issued = 0;
+      for (int idx = 0; idx < total_loads; ++idx) {
+        const int s = idx % T::NS;
+        if (!(ok = mbar_wait(bar(T::BAR_KV_EMPTY + s), ((idx / T::NS) & 1) ^ 1, abort_flag))) break;
+        mbar_arrive_expect_tx(bar(T::BAR_KV_FULL + s), T::TILE_BYTES);
+        const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
+        for (int b = 0; b < T::NBOX; ++b)
+          tma_load_3d(sbase + T::OFF_KV + s * T::TILE_BYTES + b * T::BOX_BYTES, map, bar(T::BAR_KV_FULL + s),
+                      64 * b, 128 * (idx >> 1), bh);
+        issued = idx + 1;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // Wait (bounded) for the copies still in flight before shared memory is given back.
+        const volatile int never = 0;
+        for (int idx = max(0, issued - T::NS); idx < issued; ++idx)
+          mbar_wait(bar(T::BAR_KV_FULL + idx % T::NS), (idx / T::NS) & 1, &never);
+        mbar_wait(bar(T::BAR_Q), 0, &never);
+      }
+    }
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, T::TMEM_COLS);
+  }
+}
+
+// Nk == 0: every row sees no key.
+__global__ void fa_fwd_empty_kernel(__nv_bfloat16* o, float* lse, long long rows, int D) {
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i < rows * D) o[i] = __float2bfloat16(0.f);
+  if (i < rows) lse[i] = -INFINITY;
+}
+
+}  // namespace fa

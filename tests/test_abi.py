@@ -1,0 +1,123 @@
+"""The C-ABI library: it loads, exports every call include/fa.h declares, and
+rejects bad arguments on the host before touching the GPU (no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import io_aware_exact_32_b200 as fa
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from io_aware_exact_32_b200 import build
+    build.build()
+    return fa.lib()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_decode_splitkv", "fa_decode_workspace_size",
+              "fa_get_device_error", "fa_status_string", "fa_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+
+
+def test_only_declared_symbols_are_exported():
+    out = os.popen(f"nm -D --defined-only {fa.lib_path}").read()
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert exported == set(declared_functions())
+
+
+def test_status_strings(L):
+    for code in range(7):
+        assert len(fa.fa_status_string(code)) > 0
+    assert fa.fa_version() == 100
+
+
+NULL = ctypes.c_void_p(0)
+A16 = ctypes.c_void_p(0x10000)      # fake, aligned, never dereferenced
+MIS = ctypes.c_void_p(0x10008)      # fake, misaligned
+
+
+def fwd(L, q=A16, k=A16, v=A16, o=A16, lse=A16, B=1, H=1, Nq=128, Nk=128, d=64, scale=0.125, causal=0):
+    return L.fa_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, NULL)
+
+
+def test_fwd_validation(L):
+    assert fwd(L, d=96) == 2
+    assert fwd(L, d=32) == 2
+    assert fwd(L, B=-1) == 1
+    assert fwd(L, Nq=-5) == 1
+    assert fwd(L, scale=0.0) == 1
+    assert fwd(L, scale=float("nan")) == 1
+    assert fwd(L, scale=-1.0) == 1
+    assert fwd(L, Nq=(1 << 24) + 1) == 2
+    assert fwd(L, q=NULL) == 1
+    assert fwd(L, lse=NULL) == 1
+    assert fwd(L, k=MIS) == 3
+    assert fwd(L, o=MIS) == 3
+    # empty problems are no-ops that launch nothing
+    assert fwd(L, B=0) == 0
+    assert fwd(L, H=0, q=NULL) == 0
+    assert fwd(L, Nq=0, q=NULL, o=NULL, lse=NULL) == 0
+
+
+def bwd(L, ws=A16, ws_bytes=1 << 30, d=64, Nq=128, Nk=128, mis=None, null=None):
+    args = [A16] * 9
+    if mis is not None:
+        args[mis] = MIS
+    if null is not None:
+        args[null] = NULL
+    return L.fa_bwd(*args, ws, ws_bytes, 1, 1, Nq, Nk, d, 0.125, 0, NULL)
+
+
+def test_bwd_validation(L):
+    assert bwd(L, d=80) == 2
+    assert bwd(L, null=4) == 1          # dO
+    assert bwd(L, null=5) == 1          # lse
+    assert bwd(L, mis=7) == 3           # dk
+    assert bwd(L, ws=NULL) == 4
+    assert bwd(L, ws_bytes=16) == 4
+    assert bwd(L, ws=ctypes.c_void_p(0x10010)) == 3   # workspace must be 256-byte aligned
+    assert L.fa_bwd_workspace_size(2, 8, 1024, 64) == 2 * 8 * 1024 * 4 + 2 * 8 * 1024 * 64 * 4
+    assert L.fa_bwd_workspace_size(1, 1, 3, 128) == 256 + 3 * 128 * 4 + (256 - (3 * 128 * 4) % 256) % 256
+    assert L.fa_bwd_workspace_size(1, 1, 8, 96) == 0
+
+
+def dec(L, Lmax=8192, d=128, S=0, ws_bytes=1 << 30, seq=A16, q=A16, ws=A16):
+    return L.fa_decode_splitkv(q, A16, A16, seq, Lmax, A16, A16, 2, 4, d, 0.088, S, ws, ws_bytes, NULL)
+
+
+def test_decode_validation(L):
+    assert dec(L, d=256) == 2
+    assert dec(L, Lmax=0) == 1
+    assert dec(L, S=257) == 2
+    assert dec(L, S=-1) == 1
+    assert dec(L, seq=NULL) == 1
+    assert dec(L, seq=ctypes.c_void_p(0x10002)) == 3
+    assert dec(L, q=MIS) == 3
+    assert dec(L, ws_bytes=8) == 4
+    n = L.fa_decode_workspace_size(2, 4, 8192, 128, 0)
+    assert n >= 2 * 4 * 8 * (128 + 2) * 4
+    assert L.fa_decode_workspace_size(2, 4, 8192, 128, 3) == 2 * 4 * 3 * 128 * 4 + 256
+    assert L.fa_decode_workspace_size(2, 4, 0, 128, 0) == 0
+
+
+def test_binding_rejects_bad_tensors():
+    torch = pytest.importorskip("torch")
+    q = torch.zeros(1, 1, 4, 64, dtype=torch.float32)
+    with pytest.raises(TypeError):
+        fa.fa_fwd(q, q, q, q, torch.zeros(1, 1, 4), causal=False)

@@ -1,0 +1,124 @@
+"""Backward parity: dQ, dK, dV from the CUDA path against the float64 oracle.
+
+The CUDA backward consumes the CUDA forward's O and LSE (that is the method:
+the backward recomputes P from the saved LSE).  The oracle recomputes
+everything from the inputs in float64.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from io_aware_exact_32_b200 import workloads as W
+from oracle import attention as A
+import gpu_common as gc
+from tolerances import check_grad, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _full_check(B, H, Nq, Nk, d, causal, seed, peaked=0.0):
+    x = W.make_attention_inputs(B, H, Nq, Nk, d, seed, peaked_frac=peaked)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = gc.gpu_forward(x["q"], x["k"], x["v"], causal, scale)
+    dq, dk, dv = gc.gpu_backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal, scale)
+    q, k, v, do = (gc.f64(x[n]) for n in ("q", "k", "v", "do"))
+    rq, rk, rv = A.attention_backward(q, k, v, do, scale, causal)
+    return (check_grad(gc.f64(dq), rq, "dQ"), check_grad(gc.f64(dk), rk, "dK"),
+            check_grad(gc.f64(dv), rv, "dV"))
+
+
+def test_tiny():
+    c = W.TINY
+    for causal in c.causal:
+        _full_check(c.B, c.H, c.Nq, c.Nk, c.d, causal, c.seed)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_b2_h8_n1024_d64(causal):
+    c = W.C2
+    _full_check(c.B, c.H, c.Nq, c.Nk, c.d, causal, c.seed)
+
+
+RAGGED = [
+    (1, 1, 1, 1, 64, False),
+    (1, 2, 127, 127, 64, True),
+    (1, 1, 129, 129, 128, True),
+    (2, 1, 300, 300, 128, False),
+    (1, 3, 1000, 1000, 64, True),
+    (1, 1, 200, 500, 128, True),
+    (1, 1, 500, 200, 64, True),
+    (1, 1, 500, 200, 128, False),
+    (1, 2, 384, 640, 64, False),
+    (3, 2, 256, 256, 128, True),
+    (1, 1, 513, 1025, 128, True),
+]
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,d,causal", RAGGED)
+def test_ragged_and_edge_shapes(B, H, Nq, Nk, d, causal):
+    _full_check(B, H, Nq, Nk, d, causal, seed=23 + Nq + Nk + d)
+
+
+def test_per_row_errors_small():
+    """Per-row relative error of dQ and per-key error of dK/dV stay small, not only the aggregate."""
+    x = W.make_attention_inputs(1, 2, 640, 640, 128, 31)
+    scale = 1 / math.sqrt(128)
+    o, lse = gc.gpu_forward(x["q"], x["k"], x["v"], True, scale)
+    dq, dk, dv = gc.gpu_backward(x["q"], x["k"], x["v"], o, lse, x["do"], True, scale)
+    q, k, v, do = (gc.f64(x[n]) for n in ("q", "k", "v", "do"))
+    rq, rk, rv = A.attention_backward(q, k, v, do, scale, True)
+    for g, r, name in ((gc.f64(dq), rq, "dQ"), (gc.f64(dk), rk, "dK"), (gc.f64(dv), rv, "dV")):
+        num = np.linalg.norm(g - r, axis=-1)
+        den = np.linalg.norm(r, axis=-1).mean()
+        assert num.max() / den < 0.1, name
+
+
+def test_peaked_keys_small():
+    _full_check(1, 2, 1024, 1024, 128, True, seed=8, peaked=0.02)
+
+
+def test_workspace_reuse_and_determinism_of_dk_dv():
+    """dK/dV have no atomics: two runs agree bit for bit; dQ agrees within rounding."""
+    x = W.make_attention_inputs(1, 4, 512, 512, 64, 41)
+    scale = 0.125
+    o, lse = gc.gpu_forward(x["q"], x["k"], x["v"], True, scale)
+    a = gc.gpu_backward(x["q"], x["k"], x["v"], o, lse, x["do"], True, scale)
+    b = gc.gpu_backward(x["q"], x["k"], x["v"], o, lse, x["do"], True, scale)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    assert rel_l2(gc.f64(a[0]), gc.f64(b[0])) < 1e-2
+
+
+def _sampled_check(cfg, causal, rows_per_head, seed, last_keys=64):
+    x = W.make_config_inputs(cfg)
+    scale = cfg.scale
+    o, lse = gc.gpu_forward(x["q"], x["k"], x["v"], causal, scale)
+    dq, dk, dv = gc.gpu_backward(x["q"], x["k"], x["v"], o, lse, x["do"], causal, scale)
+    dq_h, dk_h, dv_h = gc.f64(dq), gc.f64(dk), gc.f64(dv)
+    do_h = gc.f64(x["do"])
+    assert np.all(np.isfinite(dq_h)) and np.all(np.isfinite(dk_h)) and np.all(np.isfinite(dv_h))
+    for b in range(cfg.B):
+        for h in range(cfg.H):
+            q, k, v, do = (gc.f64(x[n][b, h]) for n in ("q", "k", "v", "do"))
+            rows = gc.sample_rows(cfg.Nq, rows_per_head, seed + 97 * b + h)
+            rq = A.attention_backward_q_rows(q, k, v, do, rows, scale, causal)
+            check_grad(dq_h[b, h, rows], rq, f"dQ rows [{b},{h}]")
+            keys = np.arange(cfg.Nk - last_keys, cfg.Nk)
+            rk, rv = A.attention_backward_kv_rows(q, k, v, do, keys, scale, causal)
+            check_grad(dk_h[b, h, keys], rk, f"dK last keys [{b},{h}]")
+            check_grad(dv_h[b, h, keys], rv, f"dV last keys [{b},{h}]")
+            # Properties at any size: sum_j dK_j = 0 and sum_j dV_j = sum_i dO_i.
+            rms_k = math.sqrt(np.sum(dk_h[b, h] ** 2))
+            assert np.linalg.norm(dk_h[b, h].sum(0)) <= 0.05 * rms_k + 1e-6
+            rms_v = math.sqrt(np.sum(dv_h[b, h] ** 2))
+            assert np.linalg.norm(dv_h[b, h].sum(0) - do.sum(0)) <= 0.02 * rms_v + 1e-6
+
+
+@pytest.mark.parametrize("cfg", W.SWEEP, ids=lambda c: c.name)
+def test_sweep_full_size_sampled(cfg):
+    _sampled_check(cfg, True, rows_per_head=16, seed=13)
+
+
+def test_long_context_sampled():
+    _sampled_check(W.LONG, True, rows_per_head=24, seed=17)
