@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""Benchmark of the exact fused attention path on B200; prints ONE JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Headline workload (per GPU): B=2, H=8, Nq=Nk=1024, d=64, bf16 inputs iid N(0,1);
+one step = forward + backward with the causal mask, then forward + backward
+without it, all through the C ABI.  `value` is whole-job TFLOP/s by the
+FLOP convention 4*B*H*Nq*Nk*d per forward (halved when causal) and 2.5x that
+per backward.  L2 is flushed (a 256 MiB write) before every timed step.
+
+Alongside: `e2e` (the same step through the C ABI from pinned host buffers,
+host<->device copies inside the timed region), the roofline of the dominant
+kernel, a CPU-oracle baseline, and `extra` measurements of the d=128 causal
+N=4096 forward / forward+backward and of split-KV decode (HBM GB/s).
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own shard of
+(batch, head) units (weak scaling, no collective on the data path); times are
+the max over ranks.  `--impl reference` times the float64 CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+L2_FLUSH_BYTES = 256 << 20
+
+
+# --------------------------------------------------------------------------------- host logic
+def dist_env():
+    """(rank, world, local_rank) from the torchrun environment (1 process when absent)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own shard of (batch, head) units: distinct inputs, no exchange."""
+    return base_seed + 1000 * rank
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one process)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(per_rank_units: float, world: int, max_seconds: float) -> float:
+    return per_rank_units * world / max_seconds
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = str(gpu_index)
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", self.gpu], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(seconds: float, seed: int = 1):
+    """Time the float64 oracle on whole (batch, head) slices of the headline workload.
+
+    Returns (flops_done, elapsed, heads_done, threads)."""
+    import numpy as np
+    from io_aware_exact_32_b200 import workloads as W
+    from oracle import attention as A
+    c = W.C2
+    x = W.make_attention_inputs(c.B, c.H, c.Nq, c.Nk, c.d, seed)
+    q, k, v, do = (x[n].double().numpy() for n in ("q", "k", "v", "do"))
+    per_head = sum(W.flops_forward(1, 1, c.Nq, c.Nk, c.d, cz) + W.flops_backward(1, 1, c.Nq, c.Nk, c.d, cz)
+                   for cz in (True, False))
+    t0 = time.perf_counter()
+    heads = 0
+    while True:
+        b, h = divmod(heads % (c.B * c.H), c.H)
+        for causal in (True, False):
+            A.attention_forward_head(q[b, h], k[b, h], v[b, h], c.scale, causal)
+            A.attention_backward_head(q[b, h], k[b, h], v[b, h], do[b, h], c.scale, causal)
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return per_head * heads, el, heads, blas_threads()
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from io_aware_exact_32_b200 import workloads as W
+    c = W.C2
+    for _ in range(args.warmup):
+        cpu_oracle_sample(0.0)
+    flops, secs = 0.0, 0.0
+    for _ in range(args.steps):
+        f, el, _, threads = cpu_oracle_sample(0.0)
+        flops += f
+        secs += el
+    value = flops / secs / 1e12
+    sample = (f"{args.steps} steps, each one (batch, head) slice of B={c.B} H={c.H} N={c.Nq} d={c.d}: "
+              f"forward+backward causal and non-causal in float64 numpy")
+    line = {
+        "impl": "reference", "metric": "attention fwd+bwd TFLOP/s (causal + non-causal step)", "value": value,
+        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"b{c.B}_h{c.H}_n{c.Nq}_d{c.d} fwd+bwd causal+noncausal (one head per step)",
+                   "global_batch": c.B, "seq_len": c.Nq, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------- GPU path
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import io_aware_exact_32_b200 as fa
+    from io_aware_exact_32_b200 import build, workloads as W
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    fa.lib()
+    stream = torch.cuda.current_stream()
+    peaks = measured_peaks()
+
+    c = W.C2
+    x = W.make_attention_inputs(c.B, c.H, c.Nq, c.Nk, c.d, shard_seed(c.seed, rank))
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    B, H, N, d = c.B, c.H, c.Nq, c.d
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+    out = {}
+    for causal in (True, False):
+        out[causal] = dict(o=torch.empty_like(q), lse=torch.empty(B, H, N, device=dev, dtype=torch.float32),
+                           dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v))
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    step_flops = sum(W.flops_forward(B, H, N, N, d, cz) + W.flops_backward(B, H, N, N, d, cz) for cz in (True, False))
+    calls = [("fwd_causal", True, "fwd"), ("bwd_causal", True, "bwd"), ("fwd_noncausal", False, "fwd"),
+             ("bwd_noncausal", False, "bwd")]
+    call_flops = {name: (W.flops_forward if kind == "fwd" else W.flops_backward)(B, H, N, N, d, cz)
+                  for name, cz, kind in calls}
+    launches_per_step = 2 * (1 + 3)  # fa_fwd: 1 kernel; fa_bwd: preprocess + main + dQ convert
+
+    def step(events=None):
+        for i, (name, cz, kind) in enumerate(calls):
+            o = out[cz]
+            if events is not None:
+                events[i][0].record(stream)
+            if kind == "fwd":
+                fa.fa_fwd(q, k, v, o["o"], o["lse"], cz, c.scale, stream)
+            else:
+                fa.fa_bwd(q, k, v, o["o"], do, o["lse"], o["dq"], o["dk"], o["dv"], ws, cz, c.scale, stream)
+            if events is not None:
+                events[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        flush_buf.zero_()
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_get_device_error() != 0:
+        raise RuntimeError("device-side wait timed out during warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    call_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+               for _ in range(K)]
+    clocks = ClockSampler(dev.index if world == 1 else local).start() if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for s in range(K):
+        flush_buf.zero_()
+        ev[s][0].record(stream)
+        step(call_ev[s])
+        ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    status = fa.fa_get_device_error()
+    step_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
+    total_s = reduce_max(sum(step_ms) / 1e3, world, dev)
+    value = whole_job_rate(step_flops * K, world, total_s) / 1e12
+    call_ms = {name: statistics.mean(call_ev[s][i][0].elapsed_time(call_ev[s][i][1]) for s in range(K))
+               for i, (name, _, _) in enumerate(calls)}
+
+    # ---------------------------------------------------------------- end to end from host buffers
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+    dq_, dk_, dv_, dd_ = (torch.empty_like(t) for t in (q, k, v, do))
+    host_out = {cz: {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in out[cz].items()}
+                for cz in (True, False)}
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+    d2h = sum(t.numel() * t.element_size() for cz in (True, False) for t in host_out[cz].values())
+
+    def e2e_step():
+        for dst, src in ((dq_, hq), (dk_, hk), (dv_, hv), (dd_, hdo)):
+            dst.copy_(src, non_blocking=True)
+        for name, cz, kind in calls:
+            o = out[cz]
+            if kind == "fwd":
+                fa.fa_fwd(dq_, dk_, dv_, o["o"], o["lse"], cz, c.scale, stream)
+            else:
+                fa.fa_bwd(dq_, dk_, dv_, o["o"], dd_, o["lse"], o["dq"], o["dk"], o["dv"], ws, cz, c.scale, stream)
+        for cz in (True, False):
+            for n, t in out[cz].items():
+                host_out[cz][n].copy_(t, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    for s in range(K):
+        flush_buf.zero_()
+        e2e_ev[s][0].record(stream)
+        e2e_step()
+        e2e_ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_s = reduce_max(sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3, world, dev)
+    e2e_value = whole_job_rate(step_flops * K, world, e2e_s) / 1e12
+
+    # ---------------------------------------------------------------- dominant kernel roofline
+    dom = max(call_ms, key=lambda n: call_ms[n])
+    dom_tflops = call_flops[dom] / (call_ms[dom] / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": ("fa_bwd_main_kernel<64> (whole fa_bwd call timed: preprocess + main "
+                                              "+ dQ convert)" if dom.startswith("bwd") else "fa_fwd_kernel<64>"),
+                "call": dom, "achieved": dom_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": dom_tflops / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
+                else "fallback 1590 TFLOP/s"}
+
+    extra = {}
+    if not args.no_extra:
+        extra = extra_measurements(fa, W, dev, stream, flush_buf, peaks)
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu:
+            f, el, heads, threads = cpu_oracle_sample(args.cpu_seconds)
+            cpu = {"value": f / el / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                   "sample": f"{heads} (batch, head) slices of the headline workload, fwd+bwd causal and "
+                             f"non-causal, float64 numpy, {el:.1f} s"}
+        line = {
+            "metric": "attention fwd+bwd TFLOP/s (causal + non-causal step)", "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (iid N(0,1) bf16, seeded per rank)",
+            "config": {"workload": f"b{B}_h{H}_n{N}_d{d} fwd+bwd causal+noncausal", "global_batch": B * world,
+                       "seq_len": N, "heads": H, "head_dim": d, "parallelism": f"dp{world} over (batch, head)",
+                       "l2": "flushed before every timed step (256 MiB write)"},
+            "frac_of_peak": value / world / peaks["bf16_tflops"],
+            "per_call_ms": call_ms,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * K,
+            "clocks": clk,
+            "device_status": status,
+            "extra": extra,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
+    """d=128 causal N=4096 forward and forward+backward, and split-KV decode bandwidth."""
+    import torch
+    res = {}
+    cfg = next(c for c in W.SWEEP if c.Nq == 4096 and c.d == 128)
+    x = W.make_config_inputs(cfg)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = fa.attention_forward(q, k, v, causal=True, scale=cfg.scale)
+    ws = torch.empty(fa.fa_bwd_workspace_size(cfg.B, cfg.H, cfg.Nq, cfg.d), dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(iters):
+            flush_buf.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ts) / 1e3
+
+    t_f = timed(lambda: fa.fa_fwd(q, k, v, o, lse, True, cfg.scale, stream))
+    t_b = timed(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, True, cfg.scale, stream))
+    ff = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, True)
+    fb = W.flops_backward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, True)
+    res["causal_n4096_d128"] = {"fwd_tflops": ff / t_f / 1e12, "fwd_frac": ff / t_f / 1e12 / peaks["bf16_tflops"],
+                                "bwd_tflops": fb / t_b / 1e12,
+                                "fwd_bwd_tflops": (ff + fb) / (t_f + t_b) / 1e12,
+                                "fwd_bwd_frac": (ff + fb) / (t_f + t_b) / 1e12 / peaks["bf16_tflops"],
+                                "fwd_ms": 1e3 * t_f, "bwd_ms": 1e3 * t_b}
+    del q, k, v, do, o, lse, dq, dk, dv, ws
+    dc = W.DECODE
+    xd = W.make_decode_inputs(dc.B, dc.H, dc.Lmax, dc.d, dc.lmin, dc.seed)
+    qd, kc, vc = (xd[n].to(dev) for n in ("q", "k_cache", "v_cache"))
+    seq = xd["seqlens"].to(dev)
+    od = torch.empty_like(qd)
+    lsed = torch.empty(dc.B, dc.H, device=dev, dtype=torch.float32)
+    wsd = torch.empty(fa.fa_decode_workspace_size(dc.B, dc.H, dc.Lmax, dc.d, 0), dtype=torch.uint8, device=dev)
+    t_d = timed(lambda: fa.fa_decode_splitkv(qd, kc, vc, seq, od, lsed, wsd, dc.scale, 0, stream))
+    nbytes = W.decode_bytes(xd["seqlens"], dc.H, dc.d)
+    res["decode_b32_h32_l8192_d128"] = {"gbs": nbytes / t_d / 1e9, "frac_of_measured_hbm": nbytes / t_d / 1e9 /
+                                        peaks["hbm_gbs"], "frac_of_8000": nbytes / t_d / 1e9 / 8000.0,
+                                        "ms": 1e3 * t_d, "algorithmic_bytes": nbytes}
+    return res
+
+
+CASES = ("fwd_c2", "bwd_c2", "fwd_n4096_d128", "bwd_n4096_d128", "decode")
+
+
+def run_case(args):
+    """One C-ABI call on one workload, repeated; used for single-kernel profiling."""
+    import torch
+
+    import io_aware_exact_32_b200 as fa
+    from io_aware_exact_32_b200 import build, workloads as W
+
+    build.build()
+    dev = torch.device("cuda:0")
+    stream = torch.cuda.current_stream()
+    name = args.case
+    if name == "decode":
+        dc = W.DECODE
+        xd = W.make_decode_inputs(dc.B, dc.H, dc.Lmax, dc.d, dc.lmin, dc.seed)
+        qd, kc, vc = (xd[n].to(dev) for n in ("q", "k_cache", "v_cache"))
+        seq = xd["seqlens"].to(dev)
+        od = torch.empty_like(qd)
+        lsed = torch.empty(dc.B, dc.H, device=dev, dtype=torch.float32)
+        wsd = torch.empty(fa.fa_decode_workspace_size(dc.B, dc.H, dc.Lmax, dc.d, 0), dtype=torch.uint8, device=dev)
+        fn = lambda: fa.fa_decode_splitkv(qd, kc, vc, seq, od, lsed, wsd, dc.scale, 0, stream)
+        units, unit = W.decode_bytes(xd["seqlens"], dc.H, dc.d) / 1e9, "GB/s"
+    else:
+        cfg = W.C2 if name.endswith("c2") else next(c for c in W.SWEEP if c.Nq == 4096 and c.d == 128)
+        causal = True
+        x = W.make_config_inputs(cfg)
+        q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+        o, lse = fa.attention_forward(q, k, v, causal=causal, scale=cfg.scale)
+        if name.startswith("fwd"):
+            fn = lambda: fa.fa_fwd(q, k, v, o, lse, causal, cfg.scale, stream)
+            units = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal) / 1e12
+        else:
+            ws = torch.empty(fa.fa_bwd_workspace_size(cfg.B, cfg.H, cfg.Nq, cfg.d), dtype=torch.uint8, device=dev)
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            fn = lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, causal, cfg.scale, stream)
+            units = W.flops_backward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal) / 1e12
+        unit = "TFLOP/s"
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ts)
+    print(json.dumps({"case": name, "ms": ms, "rate": units / (ms / 1e3), "unit": unit,
+                      "device_status": fa.fa_get_device_error()}), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-extra", action="store_true", help="skip the d=128 and decode side measurements")
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="time one C-ABI call on one workload (single-kernel profiling), not the contract line")
+    args = ap.parse_args(argv)
+    if args.case:
+        return run_case(args)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -7,10 +7,12 @@
 // page (section 安全 Softmax 与在线 Softmax) applied to all chunks at once.
 //
 // The pass is bound by HBM bandwidth (each K/V byte is used for one multiply-add), so it runs on
-// the CUDA cores: a producer warp streams 32-key K and V blocks into a shared-memory ring with
+// the CUDA cores: a producer warp streams 16-key K and V blocks into a shared-memory ring with
 // plain bulk copies (exactly the visible rows, nothing past seqlens[b] is read); four consumer
-// warps each take every fourth block, one lane per key for q.k and one lane per 4 (or 2) output
+// warps each take every fourth block, two lanes per key for q.k and one lane per 4 (or 2) output
 // dims for P V, each warp with its own running (m, l, acc); the four are merged in shared memory.
+// Block i lives in ring stage i % NS with NS a multiple of the consumer-warp count, so every
+// stage belongs to one warp and is consumed in order (each wait is at most one phase ahead).
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -20,11 +22,12 @@ namespace fa {
 template <int D>
 struct DecTraits {
   static_assert(D == 64 || D == 128, "head dim");
-  static constexpr int KB = 32;  // keys per block
+  static constexpr int KB = 16;  // keys per block
   static constexpr int ROW_BYTES = D * 2;
-  static constexpr int BLK_BYTES = KB * ROW_BYTES;  // 8 KB at D = 128
-  static constexpr int NS = 6;                      // ring stages (each holds a K and a V block)
+  static constexpr int BLK_BYTES = KB * ROW_BYTES;  // 4 KB at D = 128
   static constexpr int NCW = 4;                     // consumer warps
+  static constexpr int NS = 2 * NCW;                // ring stages (each holds a K and a V block)
+  static_assert(NS % NCW == 0, "each stage must belong to one consumer warp");
   static constexpr int THREADS = 32 * (NCW + 1);
   static constexpr int NCHUNK = D / 8;  // 16-byte chunks per row
   static constexpr int PER = D / 32;    // output dims per lane
@@ -116,6 +119,7 @@ __global__ void __launch_bounds__(DecTraits<D>::THREADS) fa_decode_split_kernel(
         for (int i = max(0, issued - T::NS); i < issued; ++i) mbar_wait(full(i % T::NS), (i / T::NS) & 1, &never);
       }
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------ consumers
     float m = -INFINITY, l = 0.f;
@@ -130,14 +134,16 @@ __global__ void __launch_bounds__(DecTraits<D>::THREADS) fa_decode_split_kernel(
       const int nk = min(T::KB, nkeys - i * T::KB);
       const uint8_t* kblk = smem + T::OFF_STAGE + s * 2 * T::BLK_BYTES;
       const uint8_t* vblk = kblk + T::BLK_BYTES;
-      // score of key `lane` (log2 units); chunks visited in a lane-rotated order.
-      float sc = -INFINITY;
-      if (lane < nk) {
-        float dot = 0.f;
-        const uint8_t* krow = kblk + lane * T::ROW_BYTES;
+      // Score of key (lane & 15) in log2 units: lanes l and l + 16 each take half of the row;
+      // chunks are visited in a key-rotated order so a quarter-warp hits distinct banks.
+      const int key = lane & 15;
+      const int half = lane >> 4;
+      float dot = 0.f;
+      if (key < nk) {
+        const uint8_t* krow = kblk + key * T::ROW_BYTES;
 #pragma unroll
-        for (int c = 0; c < T::NCHUNK; ++c) {
-          const int ch = (c + lane) & (T::NCHUNK - 1);
+        for (int c = 0; c < T::NCHUNK / 2; ++c) {
+          const int ch = ((c + key) & (T::NCHUNK / 2 - 1)) + half * (T::NCHUNK / 2);
           const uint4 kv = *reinterpret_cast<const uint4*>(krow + ch * 16);
           const float4 qa = *reinterpret_cast<const float4*>(qs + ch * 12);
           const float4 qb = *reinterpret_cast<const float4*>(qs + ch * 12 + 4);
@@ -150,17 +156,18 @@ __global__ void __launch_bounds__(DecTraits<D>::THREADS) fa_decode_split_kernel(
           dot = fmaf(bf16lo_to_f32(kv.w), qb.z, dot);
           dot = fmaf(bf16hi_to_f32(kv.w), qb.w, dot);
         }
-        sc = dot;
       }
+      dot += __shfl_xor_sync(0xffffffffu, dot, 16);
+      const float sc = (key < nk) ? dot : -INFINITY;  // lanes l and l + 16 hold the same score
       float mb = sc;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
+      for (int off = 8; off > 0; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
       const float m_new = fmaxf(m, mb);  // finite: the block has at least one key
       const float alpha = ex2_approx(m - m_new);
-      const float pl = (lane < nk) ? ex2_approx(sc - m_new) : 0.f;
+      const float pl = (key < nk) ? ex2_approx(sc - m_new) : 0.f;
       float ps = pl;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      for (int off = 8; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
       l = l * alpha + ps;
 #pragma unroll
       for (int e = 0; e < T::PER; ++e) acc[e] *= alpha;

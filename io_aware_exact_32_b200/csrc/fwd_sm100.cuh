@@ -20,7 +20,8 @@
 //  * exp2 with scale*log2(e) folded into one FMA; the running max is only moved (and O and l
 //    rescaled) when a row's max grows by more than 2^8, which keeps P <= 256 and is exact
 //    because O, l and LSE all use the same stale max;
-//  * P is rounded to bf16 and written over the first half of its own S columns.
+//  * P is rounded to bf16 and written over the first half of its own S columns; the row sum l
+//    accumulates the rounded values, so normalisation matches the weights actually applied.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -194,9 +195,11 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       for (int c = 0; c < 64; ++c) {
         const float e0 = ex2_approx(fmaf(s[2 * c], p.scale_log2, -base));
         const float e1 = ex2_approx(fmaf(s[2 * c + 1], p.scale_log2, -base));
-        sum0 += e0;
-        sum1 += e1;
         pk[c] = pack_bf16x2(e0, e1);
+        // l sums the bf16-rounded weights the P V product actually uses, so O stays a convex
+        // combination of V rows (this removes most of the rounding error on peaked rows).
+        sum0 += bf16lo_to_f32(pk[c]);
+        sum1 += bf16hi_to_f32(pk[c]);
       }
       l_run = l_run * alpha + (sum0 + sum1);
       tmem_st32x32b_x64(lane_addr + colS, pk);
