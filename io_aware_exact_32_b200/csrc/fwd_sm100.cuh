@@ -20,8 +20,8 @@
 //  * exp2 with scale*log2(e) folded into one FMA; the running max is only moved (and O and l
 //    rescaled) when a row's max grows by more than 2^8, which keeps P <= 256 and is exact
 //    because O, l and LSE all use the same stale max;
-//  * P is rounded to bf16 and written over the first half of its own S columns; the row sum l
-//    accumulates the rounded values, so normalisation matches the weights actually applied.
+//  * P is rounded to bf16 and written over the first half of its own S columns; O is normalised
+//    by the sum of those rounded weights, LSE by the exact fp32 sum.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
     const uint32_t colS = T::col_s(t), colO = T::col_o(t);
     int kmax = p.Nk - 1;  // last visible key of this row (inclusive)
     if (p.causal) kmax = min(kmax, row + p.Nk - p.Nq);
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f, lr_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL + t), j & 1, abort_flag));
@@ -189,19 +189,22 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
         m_run = m_tile;
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      float sum0 = 0.f, sum1 = 0.f;
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nb2 = make_float2(-base, -base);
+      // Two row sums: the exact one feeds LSE; the sum of the bf16-rounded weights that the P V
+      // product actually uses normalises O, so O stays a convex combination of V rows (this
+      // removes most of the rounding error on sharply peaked rows).
+      float2 sum_e = make_float2(0.f, 0.f), sum_r = make_float2(0.f, 0.f);
       uint32_t pk[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
-        const float e0 = ex2_approx(fmaf(s[2 * c], p.scale_log2, -base));
-        const float e1 = ex2_approx(fmaf(s[2 * c + 1], p.scale_log2, -base));
-        pk[c] = pack_bf16x2(e0, e1);
-        // l sums the bf16-rounded weights the P V product actually uses, so O stays a convex
-        // combination of V rows (this removes most of the rounding error on peaked rows).
-        sum0 += bf16lo_to_f32(pk[c]);
-        sum1 += bf16hi_to_f32(pk[c]);
+        const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, nb2);
+        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        pk[c] = pack_bf16x2(e.x, e.y);
+        sum_e = fadd2(sum_e, e);
+        sum_r = fadd2(sum_r, make_float2(bf16lo_to_f32(pk[c]), bf16hi_to_f32(pk[c])));
       }
-      l_run = l_run * alpha + (sum0 + sum1);
+      l_run = l_run * alpha + (sum_e.x + sum_e.y);
+      lr_run = lr_run * alpha + (sum_r.x + sum_r.y);
       tmem_st32x32b_x64(lane_addr + colS, pk);
       if (__any_sync(0xffffffffu, resc)) {
         // O_t still holds the sum through tile j-1: wait until PV(j-1) has landed, then scale.
@@ -224,7 +227,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (n_kv - 1) & 1, abort_flag));
     if (ok) {
       tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv = lr_run > 0.f ? 1.f / lr_run : 0.f;
       const bool in_range = row < p.Nq;
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D;
 #pragma unroll

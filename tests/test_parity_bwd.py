@@ -101,9 +101,20 @@ def _sampled_check(cfg, causal, rows_per_head, seed, last_keys=64):
     for b in range(cfg.B):
         for h in range(cfg.H):
             q, k, v, do = (gc.f64(x[n][b, h]) for n in ("q", "k", "v", "do"))
-            rows = gc.sample_rows(cfg.Nq, rows_per_head, seed + 97 * b + h)
-            rq = A.attention_backward_q_rows(q, k, v, do, rows, scale, causal)
-            check_grad(dq_h[b, h, rows], rq, f"dQ rows [{b},{h}]")
+            # Whole-tensor relative L2 of dQ, estimated by stratified sampling: every one of the
+            # first `head_rows` rows (few visible keys, so they carry most of the norm under the
+            # causal mask) plus a uniform sample of the rest, weighted by the rows it stands for.
+            head_rows = min(256, cfg.Nq)
+            first = np.arange(head_rows)
+            rest = np.random.default_rng(seed + 97 * b + h).choice(
+                np.arange(head_rows, cfg.Nq), size=min(rows_per_head, cfg.Nq - head_rows), replace=False)
+            r_first = A.attention_backward_q_rows(q, k, v, do, first, scale, causal)
+            r_rest = A.attention_backward_q_rows(q, k, v, do, np.sort(rest), scale, causal)
+            w = (cfg.Nq - head_rows) / max(len(rest), 1)
+            num = np.sum((dq_h[b, h, first] - r_first) ** 2) + w * np.sum((dq_h[b, h, np.sort(rest)] - r_rest) ** 2)
+            den = np.sum(r_first ** 2) + w * np.sum(r_rest ** 2)
+            est = math.sqrt(num / den)
+            assert est <= 2e-2, f"dQ [{b},{h}]: estimated whole-tensor rel L2 {est:.3e}"
             keys = np.arange(cfg.Nk - last_keys, cfg.Nk)
             rk, rv = A.attention_backward_kv_rows(q, k, v, do, keys, scale, causal)
             check_grad(dk_h[b, h, keys], rk, f"dK last keys [{b},{h}]")
@@ -117,8 +128,8 @@ def _sampled_check(cfg, causal, rows_per_head, seed, last_keys=64):
 
 @pytest.mark.parametrize("cfg", W.SWEEP, ids=lambda c: c.name)
 def test_sweep_full_size_sampled(cfg):
-    _sampled_check(cfg, True, rows_per_head=16, seed=13)
+    _sampled_check(cfg, True, rows_per_head=64, seed=13)
 
 
 def test_long_context_sampled():
-    _sampled_check(W.LONG, True, rows_per_head=24, seed=17)
+    _sampled_check(W.LONG, True, rows_per_head=64, seed=17)
