@@ -14,8 +14,9 @@
  *    type bf16 (IEEE bfloat16, 2 bytes), unless stated otherwise.  LSE, D and
  *    workspaces are fp32.
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *    never allocates, frees or retains device memory; it keeps one static
- *    status word per device (see fa_get_device_error).
+ *    never allocates, frees or retains device memory at call time; its module
+ *    holds one static status word per device (see fa_get_device_error) and the
+ *    fixed scratch array of fa_decode_splitkv_noalloc.
  *  - Every tensor pointer must be 16-byte aligned (the TMA engine requires it);
  *    otherwise FA_ERR_MISALIGNED is returned and nothing is launched.
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
@@ -143,6 +144,41 @@ FA_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const voi
                             const int* seqlens, int Lmax, void* o, float* lse,
                             int B, int H, int d, float scale, int num_splits,
                             void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Capacity of the library's built-in decode scratch (bytes), used only by
+ * fa_decode_splitkv_noalloc.
+ */
+#define FA_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * Split-KV decode that allocates nothing and takes no workspace.
+ *
+ * The paper has no counterpart: this is an interface convenience for callers
+ * that cannot allocate device memory themselves -- for example a plugin whose
+ * host framework owns all device memory through its own pool and forbids raw
+ * cudaMalloc, or a latency-critical serving loop in which an allocation could
+ * synchronise the device.  Such a caller still owns q, the caches, seqlens, o
+ * and lse; the per-split partials live instead in one file-scope device array
+ * of FA_DECODE_NOALLOC_SCRATCH_BYTES inside this library, which every GPU that
+ * loads the library holds until the process exits.
+ *
+ * Arguments, layouts, results and error codes are those of fa_decode_splitkv
+ * without the workspace.  If fa_decode_workspace_size(B, H, Lmax, d,
+ * num_splits) exceeds FA_DECODE_NOALLOC_SCRATCH_BYTES the call returns
+ * FA_ERR_WORKSPACE and launches nothing.
+ *
+ * The first call on each device looks up that device's address of the scratch
+ * array (cudaGetSymbolAddress, with the device current); make that first call
+ * before any stream capture.  All calls share the one array: calls whose
+ * kernels overlap on the GPU (different streams, no ordering between them)
+ * race on it and must be serialised by the caller.  Nothing needs clearing
+ * between calls: every partial is written before it is read.
+ */
+FA_API fa_status fa_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                           const int* seqlens, int Lmax, void* o, float* lse,
+                                           int B, int H, int d, float scale, int num_splits,
+                                           void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the calling device's status

@@ -7,7 +7,8 @@ and raises on a non-zero status.  PyTorch provides device memory and streams.
 
 C-ABI mirrors (same names, torch tensors in place of pointers):
     fa_fwd, fa_bwd, fa_bwd_workspace_size, fa_decode_splitkv,
-    fa_decode_workspace_size, fa_get_device_error, fa_status_string, fa_version
+    fa_decode_workspace_size, fa_decode_splitkv_noalloc, fa_get_device_error,
+    fa_status_string, fa_version
 Convenience wrappers that allocate outputs:
     attention_forward, attention_backward, decode_splitkv
 """
@@ -20,7 +21,7 @@ import os
 __all__ = [
     "FAError", "lib", "lib_path",
     "fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_decode_splitkv", "fa_decode_workspace_size",
-    "fa_get_device_error", "fa_status_string", "fa_version",
+    "fa_decode_splitkv_noalloc", "fa_get_device_error", "fa_status_string", "fa_version",
     "attention_forward", "attention_backward", "decode_splitkv",
 ]
 
@@ -60,6 +61,8 @@ def lib() -> ctypes.CDLL:
     L.fa_decode_workspace_size.restype = sz
     L.fa_decode_splitkv.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, f, i, vp, sz, vp]
     L.fa_decode_splitkv.restype = i
+    L.fa_decode_splitkv_noalloc.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, f, i, vp]
+    L.fa_decode_splitkv_noalloc.restype = i
     L.fa_get_device_error.argtypes = [vp]
     L.fa_get_device_error.restype = i
     L.fa_status_string.argtypes = [i]
@@ -173,6 +176,31 @@ def fa_decode_splitkv(q, k_cache, v_cache, seqlens, o, lse, workspace, scale=Non
     _check(lib().fa_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(o), _ptr(lse),
                                    B, H, d, _scale(scale, d), int(num_splits), _ptr(workspace), workspace.numel(),
                                    _stream_ptr(stream)), "fa_decode_splitkv")
+
+
+def fa_decode_splitkv_noalloc(q, k_cache, v_cache, seqlens, o, lse, scale=None, num_splits: int = 0,
+                              stream=None) -> None:
+    """Split-KV decode with no workspace (see include/fa.h: fa_decode_splitkv_noalloc).
+
+    For callers that cannot allocate device memory: the partials live in the
+    library's own fixed-size device scratch, shared by every call (calls that
+    overlap on the GPU race on it)."""
+    import torch
+    B, H, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query per (batch, head)")
+    Lmax = k_cache.shape[2]
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev, (B, H, Lmax, d))
+    _need(v_cache, "v_cache", torch.bfloat16, dev, (B, H, Lmax, d))
+    _need(seqlens, "seqlens", torch.int32, dev, (B,))
+    _need(o, "o", torch.bfloat16, dev, (B, H, 1, d))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev, (B, H))
+    _check(lib().fa_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(o),
+                                           _ptr(lse), B, H, d, _scale(scale, d), int(num_splits),
+                                           _stream_ptr(stream)), "fa_decode_splitkv_noalloc")
 
 
 def fa_get_device_error(stream=None) -> int:

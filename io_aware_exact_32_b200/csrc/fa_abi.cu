@@ -296,3 +296,58 @@ const char* fa_status_string(fa_status status) {
 int fa_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free split-KV decode: the partials live in a file-scope device array instead of a
+// caller workspace.  Host code must not hand the array's name to a kernel (in host code it is a
+// host-side stand-in, not a device address); it looks up each device's address once.
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoallocScratchBytes = FA_DECODE_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoallocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once per device).
+fa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                               const int* seqlens, int Lmax, void* o, float* lse, int B, int H,
+                                               int d, float scale, int num_splits, void* stream) {
+  if (B < 0 || H < 0 || num_splits < 0) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Lmax < 1 || Lmax > kMaxSeq) return Lmax < 1 ? FA_ERR_INVALID_ARG : FA_ERR_UNSUPPORTED;
+  if (num_splits > kMaxSplits) return FA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  if (BH == 0) return FA_OK;
+  if (!q || !k_cache || !v_cache || !seqlens || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+      (lse && !aligned16(lse)) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return FA_ERR_MISALIGNED;
+  if (fa_decode_workspace_size(B, H, Lmax, d, num_splits) > kNoallocScratchBytes) return FA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  const fa_status st = noalloc_scratch(&ws);
+  if (st != FA_OK) return st;
+  const int S = decode_splits(Lmax, num_splits);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode<64>(q, k_cache, v_cache, seqlens, Lmax, o, lse, (int)BH, H, scale, S, ws, s)
+                 : launch_decode<128>(q, k_cache, v_cache, seqlens, Lmax, o, lse, (int)BH, H, scale, S, ws, s);
+}
