@@ -19,7 +19,11 @@
 //   TMEM: S^T (128 cols) | dP^T (128 cols; later reused for the dQ block) | dV (d) | dK (d)
 //   SMEM: K_j, V_j (resident), a ring of (Q_i, dO_i) stages, dS^T (bf16, 128-byte swizzle)
 //   warps 0-3: one thread per key row: P, dS, dQ read-out + atomics, dK/dV epilogue
-//   warp 4: tcgen05 MMA issuer; warp 5: TMA producer.
+//   warp 4: MMA issuer A (S^T, dV: the users of the S^T/P^T columns)
+//   warp 5: MMA issuer B (dP^T, dQ, dK); warp 6: TMA producer.
+// Two issuers because one thread issues at most one 128 x N x 16 MMA every ~115 cycles
+// (measured on B200), about half the tensor-core rate at N = 128.  Barriers that must see both
+// issuers' work (S^T and dP^T ready, a Q/dO stage free, final dK/dV) count two commits.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -51,12 +55,13 @@ struct BwdTraits {
   static constexpr int BAR_DQ_FREE = BAR_S_FULL + 3;
   static constexpr int BAR_ACC_DONE = BAR_S_FULL + 4;
   static constexpr int BAR_DRAIN = BAR_S_FULL + 5;
-  static constexpr int NBAR = BAR_DRAIN + 1;
+  static constexpr int BAR_DRAIN2 = BAR_S_FULL + 6;
+  static constexpr int NBAR = BAR_DRAIN2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 224;
   static constexpr uint32_t IDESC_SQ = make_idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
   static constexpr uint32_t IDESC_DVK = make_idesc_bf16(128, D, false, true);    // P^T dO, dS^T Q
   static constexpr uint32_t IDESC_DQ = make_idesc_bf16(128, D, true, true);      // dS K
@@ -161,14 +166,15 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     mbar_init(bar(T::BAR_KV), 1);
     for (int s = 0; s < T::NS; ++s) {
       mbar_init(bar(T::BAR_QD_FULL + s), 1);
-      mbar_init(bar(T::BAR_QD_EMPTY + s), 1);
+      mbar_init(bar(T::BAR_QD_EMPTY + s), 2);  // issuer A after dV, issuer B after dK
     }
-    mbar_init(bar(T::BAR_S_FULL), 1);
+    mbar_init(bar(T::BAR_S_FULL), 2);  // issuer A after S^T, issuer B after dP^T
     mbar_init(bar(T::BAR_DS_READY), 128);
     mbar_init(bar(T::BAR_DQ_FULL), 1);
     mbar_init(bar(T::BAR_DQ_FREE), 128);
-    mbar_init(bar(T::BAR_ACC_DONE), 1);
+    mbar_init(bar(T::BAR_ACC_DONE), 2);
     mbar_init(bar(T::BAR_DRAIN), 1);
+    mbar_init(bar(T::BAR_DRAIN2), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -176,7 +182,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 5 && lane == 0) {
+  if (warp == 6 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -306,59 +312,64 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     } else {
       *abort_flag = 1;
     }
-  } else if (warp == 4) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 4 || warp == 5) {
+    // ------------------------------------------------------------------ MMA issuers A and B
+    const bool is_a = (warp == 4);
     if (lane == 0 && n_q > 0) {
       const uint32_t k_smem = sbase + T::OFF_K, v_smem = sbase + T::OFF_V, ds_smem = sbase + T::OFF_DS;
       const uint32_t tS = tmem_base + T::COL_S, tDP = tmem_base + T::COL_DP;
       const uint32_t tDV = tmem_base + T::COL_DV, tDK = tmem_base + T::COL_DK;
       auto q_smem = [&](int it) { return sbase + T::OFF_QD + (it % T::NS) * 2 * T::TILE_BYTES; };
+      const uint64_t ds_kmaj = make_sdesc_sw128(ds_smem, 16, 1024);           // dS^T as A, K-major
+      const uint64_t ds_mn = make_sdesc_sw128(ds_smem, T::BOX_BYTES, 1024);    // dS as A, MN-major
+      const uint64_t k_mn = make_sdesc_sw128(k_smem, T::BOX_BYTES, 1024);      // K as B, MN-major
       bool ok = mbar_wait(bar(T::BAR_KV), 0, abort_flag);
-      if (ok) ok = mbar_wait(bar(T::BAR_QD_FULL + 0), 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(0));                  // S^T = K Q^T
-        bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(0) + T::TILE_BYTES);  // dP^T = V dO^T
-        mma_commit(bar(T::BAR_S_FULL));
-      }
       for (int it = 0; ok && it < n_q; ++it) {
         const uint32_t qs = q_smem(it), dos = qs + T::TILE_BYTES;
-        if (!(ok = mbar_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
-        tc_fence_after();
-        // dQ_i = dS K_j -> dP^T columns (dP^T is already consumed).  A = dS (MN-major view of dS^T).
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tDP, make_sdesc_sw128(ds_smem + kk * 2048, T::BOX_BYTES, 1024),
-                 make_sdesc_sw128(k_smem + kk * 2048, T::BOX_BYTES, 1024), T::IDESC_DQ, kk > 0 ? 1u : 0u);
-        mma_commit(bar(T::BAR_DQ_FULL));
-        // dV_j += P^T dO_i  (P^T from TMEM, dO MN-major).
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tDV, tS + kk * 8, make_sdesc_sw128(dos + kk * 2048, T::BOX_BYTES, 1024), T::IDESC_DVK,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        // dK_j += dS^T Q_i  (dS^T K-major, Q MN-major); scale is applied in the epilogue.
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tDK, make_sdesc_sw128(ds_smem + (kk / 4) * T::BOX_BYTES + (kk % 4) * 32, 16, 1024),
-                 make_sdesc_sw128(qs + kk * 2048, T::BOX_BYTES, 1024), T::IDESC_DVK, (it > 0 || kk > 0) ? 1u : 0u);
-        if (it + T::NS < n_q) mma_commit(bar(T::BAR_QD_EMPTY + it % T::NS));
-        if (it + 1 < n_q) {
-          const uint32_t qn = q_smem(it + 1);
-          if (!(ok = mbar_wait(bar(T::BAR_QD_FULL + (it + 1) % T::NS), ((it + 1) / T::NS) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(bar(T::BAR_QD_FULL + it % T::NS), (it / T::NS) & 1, abort_flag))) break;
+        if (is_a) {
           tc_fence_after();
-          bwd_issue_ss_kmajor<D>(tS, k_smem, qn);  // after dV in issue order: P^T already read
-          if (!(ok = mbar_wait(bar(T::BAR_DQ_FREE), it & 1, abort_flag))) break;
-          tc_fence_after();
-          bwd_issue_ss_kmajor<D>(tDP, v_smem, qn + T::TILE_BYTES);
+          // S^T = K Q^T.  Overwrites P^T(it-1): dV(it-1) was issued earlier by this thread.
+          bwd_issue_ss_kmajor<D>(tS, k_smem, qs);
           mma_commit(bar(T::BAR_S_FULL));
+          if (!(ok = mbar_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
+          tc_fence_after();
+          // dV_j += P^T dO_i  (P^T from TMEM, dO MN-major).
+          const uint64_t do_mn = make_sdesc_sw128(dos, T::BOX_BYTES, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tDV, tS + kk * 8, do_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK, (it > 0 || kk > 0) ? 1u : 0u);
+          if (it + T::NS < n_q) mma_commit(bar(T::BAR_QD_EMPTY + it % T::NS));
+        } else {
+          // dP^T = V dO^T into the dP^T columns, once dQ(it-1) has been read out of them.
+          if (it > 0 && !(ok = mbar_wait(bar(T::BAR_DQ_FREE), (it - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          bwd_issue_ss_kmajor<D>(tDP, v_smem, dos);
+          mma_commit(bar(T::BAR_S_FULL));
+          if (!(ok = mbar_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
+          tc_fence_after();
+          // dQ_i = dS K_j -> dP^T columns (dP^T is already consumed).  A = dS (MN-major view of dS^T).
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tDP, ds_mn + (uint64_t)((kk * 2048) >> 4), k_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DQ,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(bar(T::BAR_DQ_FULL));
+          // dK_j += dS^T Q_i  (dS^T K-major, Q MN-major); scale is applied in the epilogue.
+          const uint64_t q_mn = make_sdesc_sw128(qs, T::BOX_BYTES, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(tDK, ds_kmaj + (uint64_t)(((kk / 4) * T::BOX_BYTES + (kk % 4) * 32) >> 4),
+                   q_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK, (it > 0 || kk > 0) ? 1u : 0u);
+          if (it + T::NS < n_q) mma_commit(bar(T::BAR_QD_EMPTY + it % T::NS));
         }
       }
       if (ok) mma_commit(bar(T::BAR_ACC_DONE));
       if (!ok) {
         *abort_flag = 1;
-        mma_commit(bar(T::BAR_DRAIN));
+        const int drain = is_a ? T::BAR_DRAIN : T::BAR_DRAIN2;
+        mma_commit(bar(drain));
         const volatile int never = 0;
-        mbar_wait(bar(T::BAR_DRAIN), 0, &never);
+        mbar_wait(bar(drain), 0, &never);
       }
     }
     __syncwarp();

@@ -11,14 +11,18 @@
 // B200 design (not the pages' A100/H100 kernels):
 //  * one CTA owns two 128-row query tiles (Q0, Q1) of one (batch, head) and streams 128-key
 //    K and V tiles through a shared-memory ring filled by TMA (128-byte swizzle);
-//  * one thread issues tcgen05 MMAs: S_t = Q_t K^T (both operands in shared memory) and
-//    O_t += P_t V (P_t read from tensor memory, V from shared memory), fp32 accumulators in
-//    TMEM: S0 | S1 | O0 | O1 = 128 + 128 + d + d columns;
+//  * tcgen05 MMAs: S_t = Q_t K^T (both operands in shared memory) and O_t += P_t V (P_t read
+//    from tensor memory, V from shared memory), fp32 accumulators in TMEM:
+//    S0 | S1 | O0 | O1 = 128 + 128 + d + d columns;
+//  * one issuing thread for both tiles, in the order S0 S1 PV0 S0' PV1 S1' ..., which staggers
+//    the two softmax groups (measured on B200: two independent issuers, one per tile, ran the
+//    groups in lockstep and were ~17% slower, although a lone thread issues a 128 x 128 x 16
+//    MMA only every ~115 cycles);
 //  * two softmax warpgroups, one per query tile, each thread owning one row (= one TMEM
 //    lane): while one group exponentiates its S tile, the tensor core runs the other tile's
-//    MMAs (issue order S0 S1 PV0 S0' PV1 S1' PV0' ...);
-//  * exp2 with scale*log2(e) folded into one FMA; the running max is only moved (and O and l
-//    rescaled) when a row's max grows by more than 2^8, which keeps P <= 256 and is exact
+//    MMAs;
+//  * exp2 with scale*log2(e) folded into one packed FMA; the running max is only moved (and O
+//    and l rescaled) when a row's max grows by more than 2^8, which keeps P <= 256 and is exact
 //    because O, l and LSE all use the same stale max;
 //  * P is rounded to bf16 and written over the first half of its own S columns; O is normalised
 //    by the sum of those rounded weights, LSE by the exact fp32 sum.
@@ -30,6 +34,13 @@ namespace fa {
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// One in kPolyEvery pairs of exponentials is evaluated on the FMA pipe instead of MUFU
+// (0 = all on MUFU).  Off by default: measured on B200, moving a third or a quarter of the
+// exponentials off MUFU did not shorten the forward at d = 128.
+#ifndef FA_FWD_POLY_EVERY
+#define FA_FWD_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
 
 template <int D>
 struct FwdTraits {
@@ -58,7 +69,7 @@ struct FwdTraits {
   // TMEM columns: S_t at 128 t, O_t at 256 + D t.
   static __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }
   static __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + (uint32_t)D * t; }
-  static constexpr int THREADS = 320;  // warps 0-7 softmax, 8 MMA, 9 TMA
+  static constexpr int THREADS = 320;  // warps 0-7 softmax, 8 MMA issuer, 9 TMA
   static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, false, false);
   static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, false, true);
 };
@@ -85,23 +96,47 @@ __device__ __forceinline__ int fwd_num_kv_tiles(int q0, int Nq, int Nk, int caus
 template <int D>
 __device__ __forceinline__ void fwd_issue_qk(uint32_t tmem_d, uint32_t q_smem, uint32_t k_smem) {
   using T = FwdTraits<D>;
+  const uint64_t qd = make_sdesc_sw128(q_smem, 16, 1024), kd = make_sdesc_sw128(k_smem, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * T::BOX_BYTES + (kk % 4) * 32;
-    mma_ss(tmem_d, make_sdesc_sw128(q_smem + off, 16, 1024), make_sdesc_sw128(k_smem + off, 16, 1024),
-           T::IDESC_QK, kk > 0 ? 1u : 0u);
+    // K advances 16 elements (32 bytes) inside a 128-byte swizzle row; every 4 steps, the next box.
+    const uint64_t off = (uint64_t)(((kk / 4) * T::BOX_BYTES + (kk % 4) * 32) >> 4);
+    mma_ss(tmem_d, qd + off, kd + off, T::IDESC_QK, kk > 0 ? 1u : 0u);
   }
 }
 
 template <int D>
 __device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
   using T = FwdTraits<D>;
+  const uint64_t vd = make_sdesc_sw128(v_smem, T::BOX_BYTES, 1024);
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk) {
     // 16 keys per step: P columns advance by 8 (two bf16 per 32-bit column), V rows by 16 x 128 B.
-    mma_ts(tmem_d, tmem_p + kk * 8, make_sdesc_sw128(v_smem + kk * 2048, T::BOX_BYTES, 1024), T::IDESC_PV,
+    mma_ts(tmem_d, tmem_p + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), T::IDESC_PV,
            (accumulate || kk > 0) ? 1u : 0u);
   }
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Max over 64 values with short dependency chains (three-input max, four partial chains).
+__device__ __forceinline__ float max64(const float* s) {
+  float m0 = fmax3(s[0], s[1], s[2]), m1 = fmax3(s[3], s[4], s[5]);
+  float m2 = fmax3(s[6], s[7], s[8]), m3 = fmax3(s[9], s[10], s[11]);
+#pragma unroll
+  for (int c = 12; c < 60; c += 8) {
+    m0 = fmax3(m0, s[c], s[c + 1]);
+    m1 = fmax3(m1, s[c + 2], s[c + 3]);
+    m2 = fmax3(m2, s[c + 4], s[c + 5]);
+    m3 = fmax3(m3, s[c + 6], s[c + 7]);
+  }
+  m0 = fmax3(m0, s[60], s[61]);
+  m1 = fmax3(m1, s[62], s[63]);
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
 template <int D>
@@ -163,23 +198,34 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
     int kmax = p.Nk - 1;  // last visible key of this row (inclusive)
     if (p.causal) kmax = min(kmax, row + p.Nk - p.Nq);
     float m_run = -INFINITY, l_run = 0.f, lr_run = 0.f;
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL + t), j & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld32x32b_x128_wait(lane_addr + colS, sr);
-      float* s = reinterpret_cast<float*>(sr);
+      // Load the S row in two halves; the second half's load overlaps the first half's max.
+      uint32_t sa[64], sb[64];
+      tmem_ld32x32b_x64_nowait(lane_addr + colS, sa);
+      tmem_wait_ld_x64(sa);
+      tmem_ld32x32b_x64_nowait(lane_addr + colS + 64, sb);
+      float* s = reinterpret_cast<float*>(sa);
+      float* s2 = reinterpret_cast<float*>(sb);
       const int lim = kmax - 128 * j;  // keys [0, lim] of this tile are visible
-      if (__any_sync(0xffffffffu, lim < 127)) {
+      const bool masked = __any_sync(0xffffffffu, lim < 127);
+      if (masked) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < 64; ++c)
           if (c > lim) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      const float mx_a = max64(s);
+      tmem_wait_ld_x64(sb);
+      if (masked) {
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 64; ++c)
+          if (c + 64 > lim) s2[c] = -INFINITY;
+      }
+      const float mx = fmaxf(mx_a, max64(s2));
       const float m_tile = mx * p.scale_log2;
       float alpha = 1.f;
       bool resc = false;
@@ -189,23 +235,36 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
         m_run = m_tile;
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nb2 = make_float2(-base, -base);
-      // Two row sums: the exact one feeds LSE; the sum of the bf16-rounded weights that the P V
-      // product actually uses normalises O, so O stays a convex combination of V rows (this
-      // removes most of the rounding error on sharply peaked rows).
-      float2 sum_e = make_float2(0.f, 0.f), sum_r = make_float2(0.f, 0.f);
-      uint32_t pk[64];
+      const float2 nb2 = make_float2(-base, -base);
+      // Exponentials in four chunks of 16 pairs; each chunk of P (bf16 pairs) is stored to TMEM
+      // as soon as it is ready.  Two row sums: exact (for LSE) and of the rounded weights
+      // (normalises O so it stays a convex combination of V rows).
+      float2 sum_e[2], sum_r[2];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float2 x = ffma2(make_float2(s[2 * c], s[2 * c + 1]), sc2, nb2);
-        const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-        pk[c] = pack_bf16x2(e.x, e.y);
-        sum_e = fadd2(sum_e, e);
-        sum_r = fadd2(sum_r, make_float2(bf16lo_to_f32(pk[c]), bf16hi_to_f32(pk[c])));
+      for (int i = 0; i < 2; ++i) sum_e[i] = sum_r[i] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        const float* src = (ch < 2) ? s + 32 * ch : s2 + 32 * (ch - 2);
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float2 x = ffma2(make_float2(src[2 * c], src[2 * c + 1]), sc2, nb2);
+          float2 e;
+          if (kPolyEvery > 0 && (c % kPolyEvery) == kPolyEvery - 1) {
+            e = exp2_poly2(x);
+          } else {
+            e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          }
+          pk[c] = pack_bf16x2(e.x, e.y);
+          sum_e[c & 1] = fadd2(sum_e[c & 1], e);
+          sum_r[c & 1] = fadd2(sum_r[c & 1], make_float2(bf16lo_to_f32(pk[c]), bf16hi_to_f32(pk[c])));
+        }
+        tmem_st32x32b_x16(lane_addr + colS + 16 * ch, pk);
       }
-      l_run = l_run * alpha + (sum_e.x + sum_e.y);
-      lr_run = lr_run * alpha + (sum_r.x + sum_r.y);
-      tmem_st32x32b_x64(lane_addr + colS, pk);
+      const float2 tot_e = fadd2(sum_e[0], sum_e[1]);
+      const float2 tot_r = fadd2(sum_r[0], sum_r[1]);
+      l_run = l_run * alpha + (tot_e.x + tot_e.y);
+      lr_run = lr_run * alpha + (tot_r.x + tot_r.y);
       if (__any_sync(0xffffffffu, resc)) {
         // O_t still holds the sum through tile j-1: wait until PV(j-1) has landed, then scale.
         ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (j - 1) & 1, abort_flag));

@@ -57,20 +57,26 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// Suspend-time hint for try_wait: a waiting thread sleeps in hardware (issuing nothing) until the
+// phase completes or this many nanoseconds pass, so waiting warps do not steal issue slots from
+// the warps that share their scheduler.
+constexpr uint32_t kSuspendHintNs = 500000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
 
 // Waits for completion of the phase with the given parity.  Gives up (returns
-// false) after kWaitLimitNs, or as soon as *abort is set by another warp.
+// false) after kWaitLimitNs, or once *abort is set by another warp (checked each
+// time a suspended try_wait returns without completion).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
@@ -196,28 +202,58 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
 // ---------------------------------------------------------------------------------------------
 #include "tmem_ldst.inc"
 
-// Packed fp32 pairs (sm_100): one instruction operates on two lanes' worth of fp32 values.
+// Packed fp32 pairs (sm_100): one instruction operates on two fp32 values held in a register pair.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
-        "l"(*reinterpret_cast<uint64_t*>(&c)));
-  return *reinterpret_cast<float2*>(&d);
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
 }
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  uint64_t d;
-  asm("add.f32x2 %0, %1, %2;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
-  return *reinterpret_cast<float2*>(&d);
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
 }
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
-  uint64_t d;
-  asm("mul.f32x2 %0, %1, %2;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
-  return *reinterpret_cast<float2*>(&d);
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x on the FMA pipe for a pair of values (frees the MUFU unit, which the exponentials of the
+// softmax otherwise saturate).  Cody-Waite style range reduction: x = n + f with n = round(x)
+// obtained by adding 1.5 * 2^23 (which leaves round(x) in the low mantissa bits) and
+// f in [-0.5, 0.5]; 2^f from a cubic fitted to 2^f on [-0.5, 0.5] by iteratively reweighted
+// least squares on the relative error (our own fit; max relative error 7.5e-5 in fp32 Horner
+// form, far below the 2^-9 of the bf16 rounding that follows); 2^n is added to the exponent
+// field.  Inputs below -125 (including -inf) return exactly 0: they are clamped first so the
+// exponent field cannot wrap, then zeroed.  Valid for x <= 127.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992812f, c1 = 0.69326097f, c2 = 0.24261054f, c3 = 0.05517132f;
+  const bool zx = x.x < -125.f, zy = x.y < -125.f;
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+  p = ffma2(p, f, make_float2(c1, c1));
+  p = ffma2(p, f, make_float2(c0, c0));
+  const uint32_t bx = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
+  const uint32_t by = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
+  return make_float2(zx ? 0.f : __uint_as_float(bx), zy ? 0.f : __uint_as_float(by));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
