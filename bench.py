@@ -315,11 +315,18 @@ def run_ours(args):
     e2e_value = whole_job_rate(step_flops * K, world, e2e_s) / 1e12
 
     # ---------------------------------------------------------------- dominant kernel roofline
-    dom = max(call_ms, key=lambda n: call_ms[n])
-    dom_tflops = call_flops[dom] / (call_ms[dom] / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": ("fa_bwd_main_kernel<64> (whole fa_bwd call timed: preprocess + main "
-                                              "+ dQ convert)" if dom.startswith("bwd") else "fa_fwd_kernel<64>"),
-                "call": dom, "achieved": dom_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+    # The kernel with the most time per step (fa_bwd_main_kernel, in both mask modes) is timed per
+    # fa_bwd call; the call also holds the two small preprocess / dQ-convert kernels, so the
+    # achieved rate understates the main kernel slightly.
+    kind_ms = {k: sum(call_ms[n] for n, _, kk in calls if kk == k) for k in ("fwd", "bwd")}
+    dom = max(kind_ms, key=lambda k: kind_ms[k])
+    dom_flops = sum(call_flops[n] for n, _, kk in calls if kk == dom)
+    dom_tflops = dom_flops / (kind_ms[dom] / 1e3) / 1e12
+    roofline = {"bound": "tensor",
+                "kernel": ("fa_bwd_main_kernel<64>, timed per fa_bwd call (with its preprocess and dQ-convert "
+                           "kernels), causal + non-causal" if dom == "bwd"
+                           else "fa_fwd_kernel<64>, causal + non-causal"),
+                "achieved": dom_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": dom_tflops / peaks["bf16_tflops"], "traffic": None,
                 "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
                 else "fallback 1590 TFLOP/s"}
