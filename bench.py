@@ -5,7 +5,9 @@
 
 Headline workload (per GPU): B=2, H=8, Nq=Nk=1024, d=64, bf16 inputs iid N(0,1);
 one step = forward + backward with the causal mask, then forward + backward
-without it, all through the C ABI.  `value` is whole-job TFLOP/s by the
+without it, all through the C ABI, captured once as a CUDA graph and replayed
+for every timed step (`--no-graph`: eager launches; the eager rate is reported
+beside it either way).  `value` is whole-job TFLOP/s by the
 FLOP convention 4*B*H*Nq*Nk*d per forward (halved when causal) and 2.5x that
 per backward.  L2 is flushed (a 256 MiB write) before every timed step.
 
@@ -235,17 +237,18 @@ def run_ours(args):
                   for name, cz, kind in calls}
     launches_per_step = 2 * (1 + 3)  # fa_fwd: 1 kernel; fa_bwd: preprocess + main + dQ convert
 
-    def step(events=None):
+    def step(events=None, st=None):
+        st = stream if st is None else st
         for i, (name, cz, kind) in enumerate(calls):
             o = out[cz]
             if events is not None:
-                events[i][0].record(stream)
+                events[i][0].record(st)
             if kind == "fwd":
-                fa.fa_fwd(q, k, v, o["o"], o["lse"], cz, c.scale, stream)
+                fa.fa_fwd(q, k, v, o["o"], o["lse"], cz, c.scale, st)
             else:
-                fa.fa_bwd(q, k, v, o["o"], do, o["lse"], o["dq"], o["dk"], o["dv"], ws, cz, c.scale, stream)
+                fa.fa_bwd(q, k, v, o["o"], do, o["lse"], o["dq"], o["dk"], o["dv"], ws, cz, c.scale, st)
             if events is not None:
-                events[i][1].record(stream)
+                events[i][1].record(st)
 
     for _ in range(args.warmup):
         flush_buf.zero_()
@@ -254,10 +257,23 @@ def run_ours(args):
     if fa.fa_get_device_error() != 0:
         raise RuntimeError("device-side wait timed out during warm-up")
 
+    # One step captured as a CUDA graph (the launch-bound inner loop: 8 small kernel launches);
+    # every timed iteration replays it, with the L2 flush and the events outside the graph.
+    graph = None
+    if not args.no_graph:
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            step(st=cap)
+        stream.wait_stream(cap)
+        for _ in range(args.warmup):
+            flush_buf.zero_()
+            graph.replay()
+        torch.cuda.synchronize()
+
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    call_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
-               for _ in range(K)]
     clocks = ClockSampler(dev.index if world == 1 else local).start() if rank == 0 else None
     if world > 1:
         dist.barrier()
@@ -265,7 +281,10 @@ def run_ours(args):
     for s in range(K):
         flush_buf.zero_()
         ev[s][0].record(stream)
-        step(call_ev[s])
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
         ev[s][1].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -275,8 +294,22 @@ def run_ours(args):
     step_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
     total_s = reduce_max(sum(step_ms) / 1e3, world, dev)
     value = whole_job_rate(step_flops * K, world, total_s) / 1e12
-    call_ms = {name: statistics.mean(call_ev[s][i][0].elapsed_time(call_ev[s][i][1]) for s in range(K))
+
+    # Per-call device times (eager launches, events around each C-ABI call) for the roofline.
+    Kc = min(K, 500)
+    call_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+               for _ in range(Kc)]
+    eager_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Kc)]
+    for s in range(Kc):
+        flush_buf.zero_()
+        eager_ev[s][0].record(stream)
+        step(call_ev[s])
+        eager_ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    call_ms = {name: statistics.mean(call_ev[s][i][0].elapsed_time(call_ev[s][i][1]) for s in range(Kc))
                for i, (name, _, _) in enumerate(calls)}
+    eager_s = reduce_max(sum(a.elapsed_time(b) for a, b in eager_ev) / 1e3, world, dev)
+    value_eager = whole_job_rate(step_flops * Kc, world, eager_s) / 1e12
 
     # ---------------------------------------------------------------- end to end from host buffers
     hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
@@ -351,7 +384,9 @@ def run_ours(args):
             "data": "synthetic (iid N(0,1) bf16, seeded per rank)",
             "config": {"workload": f"b{B}_h{H}_n{N}_d{d} fwd+bwd causal+noncausal", "global_batch": B * world,
                        "seq_len": N, "heads": H, "head_dim": d, "parallelism": f"dp{world} over (batch, head)",
-                       "l2": "flushed before every timed step (256 MiB write)"},
+                       "l2": "flushed before every timed step (256 MiB write)",
+                       "launch": "CUDA graph of one step, replayed" if graph is not None else "eager"},
+            "value_eager_launches": value_eager,
             "frac_of_peak": value / world / peaks["bf16_tflops"],
             "per_call_ms": call_ms,
             "roofline": roofline,
@@ -486,6 +521,7 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-extra", action="store_true", help="skip the d=128 and decode side measurements")
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of a replayed CUDA graph")
     ap.add_argument("--case", choices=CASES, default=None,
                     help="time one C-ABI call on one workload (single-kernel profiling), not the contract line")
     args = ap.parse_args(argv)

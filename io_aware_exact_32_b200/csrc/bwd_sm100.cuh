@@ -16,14 +16,21 @@
 //
 // Main-kernel layout (computed transposed, keys on TMEM lanes, so that dK/dV rows and the
 // P^T operand of dV = P^T dO live on the lane that owns the key):
-//   TMEM: S^T (128 cols) | dP^T (128 cols; later reused for the dQ block) | dV (d) | dK (d)
-//   SMEM: K_j, V_j (resident), a ring of (Q_i, dO_i) stages, dS^T (bf16, 128-byte swizzle)
-//   warps 0-3: one thread per key row: P, dS, dQ read-out + atomics, dK/dV epilogue
-//   warp 4: MMA issuer A (S^T, dV: the users of the S^T/P^T columns)
-//   warp 5: MMA issuer B (dP^T, dQ, dK); warp 6: TMA producer.
+//   TMEM: S^T (128 cols) | dP^T (128 cols) | dV (d) | dK (d) | dQ (d = 64 only; at d = 128 the
+//         dQ block reuses the dP^T columns once dP^T has been consumed)
+//   SMEM: K_j, V_j (resident), a ring of (Q_i, dO_i) stages, dS^T (bf16, 128-byte swizzle),
+//         and at d = 64 an fp32 staging tile for the dQ block
+//   warps 0-3: one thread per key row: P, dS (the critical path), dK/dV epilogue
+//   warps 4-7: one thread per query row of the dQ block: read it out of TMEM, release the
+//              columns at once, then add it into the fp32 accumulator (d = 64: one TMA bulk
+//              reduce-add of the staged tile; d = 128: per-thread atomics)
+//   warp 8: MMA issuer A (S^T, dV: the users of the S^T/P^T columns)
+//   warp 9: MMA issuer B (dP^T, dQ, dK); warp 10: TMA producer.
 // Two issuers because one thread issues at most one 128 x N x 16 MMA every ~115 cycles
-// (measured on B200), about half the tensor-core rate at N = 128.  Barriers that must see both
-// issuers' work (S^T and dP^T ready, a Q/dO stage free, final dK/dV) count two commits.
+// (measured on B200), about half the tensor-core rate at N = 128.  Each issuer runs one
+// iteration ahead: right after the MMAs that consume block i it issues the next block's S^T /
+// dP^T, so the compute warps wait only for those.  Barriers that must see both issuers' work
+// (S^T and dP^T ready, a Q/dO stage free, final dK/dV) count two commits.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -35,6 +42,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 template <int D>
 struct BwdTraits {
   static_assert(D == 64 || D == 128, "head dim");
+  static constexpr bool SEP_DQ = (D == 64);            // dQ block has its own TMEM columns + TMA reduce
   static constexpr int NBOX = D / 64;
   static constexpr int BOX_BYTES = 128 * 64 * 2;       // 16 KB
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // 128 x D bf16
@@ -43,25 +51,30 @@ struct BwdTraits {
   static constexpr int OFF_V = TILE_BYTES;
   static constexpr int OFF_QD = 2 * TILE_BYTES;              // stage s: Q at +0, dO at +TILE_BYTES
   static constexpr int OFF_DS = OFF_QD + NS * 2 * TILE_BYTES;  // 128 keys x 128 queries bf16 = 32 KB
-  static constexpr int OFF_STAT = OFF_DS + 2 * BOX_BYTES;      // [2][128] fp32: LSE*log2e, D
+  static constexpr int OFF_STG = OFF_DS + 2 * BOX_BYTES;       // dQ staging, 2 x (128 rows x 32 fp32) (d = 64)
+  static constexpr int STG_BYTES = SEP_DQ ? 128 * 64 * 4 : 0;
+  static constexpr int OFF_STAT = OFF_STG + STG_BYTES;         // [2][128] fp32: LSE*log2e, D
   static constexpr int OFF_BAR = OFF_STAT + 2 * 128 * 4;
-  // barriers: kv_full | qd_full[NS] | qd_empty[NS] | s_full | ds_ready | dq_full | dq_free | acc_done | drain
+  // barriers: kv_full | qd_full[NS] | qd_empty[NS] | s_full | ds_ready | ds_free | dq_full | dq_free |
+  //           acc_done | drain A | drain B
   static constexpr int BAR_KV = 0;
   static constexpr int BAR_QD_FULL = 1;
   static constexpr int BAR_QD_EMPTY = 1 + NS;
   static constexpr int BAR_S_FULL = 1 + 2 * NS;
   static constexpr int BAR_DS_READY = BAR_S_FULL + 1;
-  static constexpr int BAR_DQ_FULL = BAR_S_FULL + 2;
-  static constexpr int BAR_DQ_FREE = BAR_S_FULL + 3;
-  static constexpr int BAR_ACC_DONE = BAR_S_FULL + 4;
-  static constexpr int BAR_DRAIN = BAR_S_FULL + 5;
-  static constexpr int BAR_DRAIN2 = BAR_S_FULL + 6;
+  static constexpr int BAR_DS_FREE = BAR_S_FULL + 2;
+  static constexpr int BAR_DQ_FULL = BAR_S_FULL + 3;
+  static constexpr int BAR_DQ_FREE = BAR_S_FULL + 4;
+  static constexpr int BAR_ACC_DONE = BAR_S_FULL + 5;
+  static constexpr int BAR_DRAIN = BAR_S_FULL + 6;
+  static constexpr int BAR_DRAIN2 = BAR_S_FULL + 7;
   static constexpr int NBAR = BAR_DRAIN2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
-  static constexpr int THREADS = 224;
+  static constexpr uint32_t COL_DQ = SEP_DQ ? 256 + 2 * D : COL_DP;
+  static constexpr int THREADS = 352;
   static constexpr uint32_t IDESC_SQ = make_idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
   static constexpr uint32_t IDESC_DVK = make_idesc_bf16(128, D, false, true);    // P^T dO, dS^T Q
   static constexpr uint32_t IDESC_DQ = make_idesc_bf16(128, D, true, true);      // dS K
@@ -132,19 +145,31 @@ __device__ __forceinline__ int bwd_first_q_tile(int k0, int Nq, int Nk, int caus
 template <int D>
 __device__ __forceinline__ void bwd_issue_ss_kmajor(uint32_t tmem_d, uint32_t a_smem, uint32_t b_smem) {
   using T = BwdTraits<D>;
+  const uint64_t ad = make_sdesc_sw128(a_smem, 16, 1024), bd = make_sdesc_sw128(b_smem, 16, 1024);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * T::BOX_BYTES + (kk % 4) * 32;
-    mma_ss(tmem_d, make_sdesc_sw128(a_smem + off, 16, 1024), make_sdesc_sw128(b_smem + off, 16, 1024),
-           T::IDESC_SQ, kk > 0 ? 1u : 0u);
+    const uint64_t off = (uint64_t)(((kk / 4) * T::BOX_BYTES + (kk % 4) * 32) >> 4);
+    mma_ss(tmem_d, ad + off, bd + off, T::IDESC_SQ, kk > 0 ? 1u : 0u);
   }
 }
+
+// TMA bulk reduce-add of a staged shared-memory tile into global memory (tensor map coordinates).
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 template <int D>
 __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                       const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using T = BwdTraits<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -170,6 +195,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     }
     mbar_init(bar(T::BAR_S_FULL), 2);  // issuer A after S^T, issuer B after dP^T
     mbar_init(bar(T::BAR_DS_READY), 128);
+    mbar_init(bar(T::BAR_DS_FREE), 1);  // issuer B after dQ and dK (the readers of dS^T)
     mbar_init(bar(T::BAR_DQ_FULL), 1);
     mbar_init(bar(T::BAR_DQ_FREE), 128);
     mbar_init(bar(T::BAR_ACC_DONE), 2);
@@ -178,15 +204,16 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 6 && lane == 0) {
+  if (warp == 10 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmDO);
+    if (T::SEP_DQ) tma_prefetch_desc(&tmDQ);
   }
   tc_fence_before();
   __syncthreads();
@@ -194,8 +221,8 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp < 4) {
-    // ------------------------------------------------------------------ compute warpgroup
-    const int r = warp * 32 + lane;  // key row in the block == TMEM lane; also the dQ query row
+    // ------------------------------------------------------------------ P / dS warpgroup
+    const int r = warp * 32 + lane;  // key row in the block == TMEM lane
     const int key = k0 + r;
     const bool key_ok = key < p.Nk;
     const uint32_t lane_addr = tmem_base + ((uint32_t)(warp * 32) << 16);
@@ -226,8 +253,9 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
 #pragma unroll 1
       for (int c32 = 0; c32 < 4; ++c32) {
         uint32_t sv[32], dpv[32];
-        tmem_ld32x32b_x32_wait(lane_addr + T::COL_S + 32 * c32, sv);
-        tmem_ld32x32b_x32_wait(lane_addr + T::COL_DP + 32 * c32, dpv);
+        tmem_ld32x32b_x32_nowait(lane_addr + T::COL_S + 32 * c32, sv);
+        tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DP + 32 * c32, dpv);
+        tmem_wait_ld_2x32(sv, dpv);
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
@@ -240,8 +268,14 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           pk[i / 2] = pack_bf16x2(p0, p1);
           dk[i / 2] = pack_bf16x2(d0, d1);
         }
-        // P^T chunk -> TMEM (first 64 columns of the S^T block, bf16 pairs).
+        // P^T chunk -> TMEM (first 64 columns of the S^T block, bf16 pairs).  The S^T columns
+        // are free: S_FULL also covers issuer A's dV(it-1), the reader of P^T(it-1).
         tmem_st32x32b_x16(lane_addr + T::COL_S + 16 * c32, pk);
+        // dS^T(it-1) must have been read by dQ(it-1) and dK(it-1) before it is overwritten.
+        if (c32 == 0 && it > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DS_FREE), (it - 1) & 1, abort_flag));
+          if (!ok) break;
+        }
         // dS^T chunk -> shared memory, K-major with 128-byte swizzle (box = 64 query columns).
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -252,33 +286,11 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
                        : "memory");
         }
       }
+      if (!ok) break;
       tmem_st_wait();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(T::BAR_DS_READY));
-      // dQ block (query rows on lanes) -> scale -> atomic add into the fp32 accumulator.
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DQ_FULL), it & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      {
-        const int q = q0 + r;
-        float* dst = p.dq_acc + ((size_t)bh * p.Nq + (q < p.Nq ? q : 0)) * D;
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32x32b_x32_wait(lane_addr + T::COL_DP + 32 * c, v);
-          if (q < p.Nq) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float4 a = make_float4(__uint_as_float(v[4 * i]) * p.scale, __uint_as_float(v[4 * i + 1]) * p.scale,
-                                     __uint_as_float(v[4 * i + 2]) * p.scale, __uint_as_float(v[4 * i + 3]) * p.scale);
-              atomicAdd(reinterpret_cast<float4*>(dst + 32 * c + 4 * i), a);
-            }
-          }
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(bar(T::BAR_DQ_FREE));
     }
     // dK, dV epilogue.
     if (ok && n_q > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_ACC_DONE), 0, abort_flag));
@@ -312,54 +324,131 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     } else {
       *abort_flag = 1;
     }
-  } else if (warp == 4 || warp == 5) {
+  } else if (warp < 8) {
+    // ------------------------------------------------------------------ dQ warpgroup
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // query row of the dQ block == TMEM lane
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const bool leader = (warp == 4 && lane == 0);
+    const uint32_t stg_row = sbase + T::OFF_STG + r * 128;
+    bool ok = true;
+    for (int it = 0; it < n_q; ++it) {
+      const int q0 = (i0 + it) * 128;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DQ_FULL), it & 1, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v[D];
+      if constexpr (D == 128) {
+        tmem_ld32x32b_x128_nowait(lane_addr + T::COL_DQ, v);
+        tmem_wait_ld_x128(v);
+      } else {
+        tmem_ld32x32b_x64_nowait(lane_addr + T::COL_DQ, v);
+        tmem_wait_ld_x64(v);
+      }
+      // The dQ columns are free as soon as they are in registers.
+      tc_fence_before();
+      mbar_arrive(bar(T::BAR_DQ_FREE));
+      if constexpr (T::SEP_DQ) {
+        // Stage the scaled block as two 32-column fp32 boxes in the 128-byte-swizzle layout (row r
+        // at r*128 bytes of each box, 16-byte chunk c at (c ^ r%8)*16: a quarter-warp hits
+        // distinct banks), then bulk reduce-add both boxes.
+        if (it > 0) {
+          if (leader) bulk_wait_group_read0();  // previous tile read out of the staging buffer
+          asm volatile("bar.sync 2, 128;" ::: "memory");
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint32_t addr = stg_row + (c >> 3) * (128 * 128) + (((c & 7) ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "f"(__uint_as_float(v[4 * c]) * p.scale), "f"(__uint_as_float(v[4 * c + 1]) * p.scale),
+                       "f"(__uint_as_float(v[4 * c + 2]) * p.scale), "f"(__uint_as_float(v[4 * c + 3]) * p.scale)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        if (leader) {
+          // Rows past Nq fall outside the tensor map and are not written.
+          tma_reduce_add_3d(&tmDQ, sbase + T::OFF_STG, 0, q0, bh);
+          tma_reduce_add_3d(&tmDQ, sbase + T::OFF_STG + 128 * 128, 32, q0, bh);
+          bulk_commit_group();
+        }
+      } else {
+        const int q = q0 + r;
+        if (q < p.Nq) {
+          float* dst = p.dq_acc + ((size_t)bh * p.Nq + q) * D;
+#pragma unroll
+          for (int i = 0; i < D / 4; ++i) {
+            float4 a = make_float4(__uint_as_float(v[4 * i]) * p.scale, __uint_as_float(v[4 * i + 1]) * p.scale,
+                                   __uint_as_float(v[4 * i + 2]) * p.scale, __uint_as_float(v[4 * i + 3]) * p.scale);
+            atomicAdd(reinterpret_cast<float4*>(dst + 4 * i), a);
+          }
+        }
+      }
+    }
+    if (!ok) *abort_flag = 1;
+    if (T::SEP_DQ && leader) bulk_wait_group0();  // every reduce-add complete before the CTA exits
+  } else if (warp == 8 || warp == 9) {
     // ------------------------------------------------------------------ MMA issuers A and B
-    const bool is_a = (warp == 4);
+    const bool is_a = (warp == 8);
     if (lane == 0 && n_q > 0) {
       const uint32_t k_smem = sbase + T::OFF_K, v_smem = sbase + T::OFF_V, ds_smem = sbase + T::OFF_DS;
-      const uint32_t tS = tmem_base + T::COL_S, tDP = tmem_base + T::COL_DP;
+      const uint32_t tS = tmem_base + T::COL_S, tDP = tmem_base + T::COL_DP, tDQ = tmem_base + T::COL_DQ;
       const uint32_t tDV = tmem_base + T::COL_DV, tDK = tmem_base + T::COL_DK;
       auto q_smem = [&](int it) { return sbase + T::OFF_QD + (it % T::NS) * 2 * T::TILE_BYTES; };
+      auto wait_qd = [&](int it) { return mbar_wait(bar(T::BAR_QD_FULL + it % T::NS), (it / T::NS) & 1, abort_flag); };
       const uint64_t ds_kmaj = make_sdesc_sw128(ds_smem, 16, 1024);           // dS^T as A, K-major
       const uint64_t ds_mn = make_sdesc_sw128(ds_smem, T::BOX_BYTES, 1024);    // dS as A, MN-major
       const uint64_t k_mn = make_sdesc_sw128(k_smem, T::BOX_BYTES, 1024);      // K as B, MN-major
-      bool ok = mbar_wait(bar(T::BAR_KV), 0, abort_flag);
+      bool ok = mbar_wait(bar(T::BAR_KV), 0, abort_flag) && wait_qd(0);
+      if (ok) {
+        tc_fence_after();
+        if (is_a) bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(0));                   // S^T = K Q^T
+        else bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(0) + T::TILE_BYTES);       // dP^T = V dO^T
+        mma_commit(bar(T::BAR_S_FULL));
+      }
       for (int it = 0; ok && it < n_q; ++it) {
         const uint32_t qs = q_smem(it), dos = qs + T::TILE_BYTES;
-        if (!(ok = mbar_wait(bar(T::BAR_QD_FULL + it % T::NS), (it / T::NS) & 1, abort_flag))) break;
+        const bool more = it + 1 < n_q;
+        if (!(ok = mbar_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
+        tc_fence_after();
         if (is_a) {
-          tc_fence_after();
-          // S^T = K Q^T.  Overwrites P^T(it-1): dV(it-1) was issued earlier by this thread.
-          bwd_issue_ss_kmajor<D>(tS, k_smem, qs);
-          mma_commit(bar(T::BAR_S_FULL));
-          if (!(ok = mbar_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
-          tc_fence_after();
-          // dV_j += P^T dO_i  (P^T from TMEM, dO MN-major).
+          // dV_j += P^T dO_i  (P^T from TMEM, dO MN-major); then the next block's S^T, which
+          // overwrites P^T(it) only after dV(it) (same issuing thread, executed in order).
           const uint64_t do_mn = make_sdesc_sw128(dos, T::BOX_BYTES, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tDV, tS + kk * 8, do_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK, (it > 0 || kk > 0) ? 1u : 0u);
           if (it + T::NS < n_q) mma_commit(bar(T::BAR_QD_EMPTY + it % T::NS));
+          if (more) {
+            if (!(ok = wait_qd(it + 1))) break;
+            tc_fence_after();
+            bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(it + 1));
+            mma_commit(bar(T::BAR_S_FULL));
+          }
         } else {
-          // dP^T = V dO^T into the dP^T columns, once dQ(it-1) has been read out of them.
-          if (it > 0 && !(ok = mbar_wait(bar(T::BAR_DQ_FREE), (it - 1) & 1, abort_flag))) break;
+          // dQ_i = dS K_j (A = dS, the MN-major view of dS^T), once the dQ columns are free.
+          if (T::SEP_DQ && it > 0 && !(ok = mbar_wait(bar(T::BAR_DQ_FREE), (it - 1) & 1, abort_flag))) break;
           tc_fence_after();
-          bwd_issue_ss_kmajor<D>(tDP, v_smem, dos);
-          mma_commit(bar(T::BAR_S_FULL));
-          if (!(ok = mbar_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
-          tc_fence_after();
-          // dQ_i = dS K_j -> dP^T columns (dP^T is already consumed).  A = dS (MN-major view of dS^T).
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDP, ds_mn + (uint64_t)((kk * 2048) >> 4), k_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DQ,
+            mma_ss(tDQ, ds_mn + (uint64_t)((kk * 2048) >> 4), k_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DQ,
                    kk > 0 ? 1u : 0u);
           mma_commit(bar(T::BAR_DQ_FULL));
+          // Next block's dP^T (at d = 128 it reuses the dQ columns: wait until dQ(it) is read out).
+          if (more) {
+            if (!(ok = wait_qd(it + 1))) break;
+            if (!T::SEP_DQ && !(ok = mbar_wait(bar(T::BAR_DQ_FREE), it & 1, abort_flag))) break;
+            tc_fence_after();
+            bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(it + 1) + T::TILE_BYTES);
+            mma_commit(bar(T::BAR_S_FULL));
+          }
           // dK_j += dS^T Q_i  (dS^T K-major, Q MN-major); scale is applied in the epilogue.
           const uint64_t q_mn = make_sdesc_sw128(qs, T::BOX_BYTES, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss(tDK, ds_kmaj + (uint64_t)(((kk / 4) * T::BOX_BYTES + (kk % 4) * 32) >> 4),
                    q_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK, (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(T::BAR_DS_FREE));
           if (it + T::NS < n_q) mma_commit(bar(T::BAR_QD_EMPTY + it % T::NS));
         }
       }
@@ -408,7 +497,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem_base, T::TMEM_COLS);
   }

@@ -50,6 +50,21 @@ bool make_map_3d(CUtensorMap* map, const void* base, int D, int N, long long BH)
   return r == CUDA_SUCCESS;
 }
 
+// [BH, N, D] fp32 viewed as {D, N, BH}; box = 32 columns x 128 rows x 1, 128-byte swizzle (the dQ
+// accumulator, target of the backward's bulk reduce-add).  Rows past N are not written.
+bool make_map_3d_f32(CUtensorMap* map, void* base, int D, int N, long long BH) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)N * D * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -68,6 +83,19 @@ bool set_smem(K kernel, int bytes) {
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
   if (ndone[dev] < 16) done[dev][ndone[dev]++] = reinterpret_cast<const void*>(kernel);
   return true;
+}
+
+// Multiprocessor count of the current device (cached per device).
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
 }
 
 fa_status check_common(int B, int H, int Nq, int Nk, int d, float scale) {
@@ -104,10 +132,12 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   p.Nq = Nq;
   p.Nk = Nk;
   p.BH = BH;
-  p.npairs = (Nq + 255) / 256;
+  // Two 128-row tiles per CTA (softmax / MMA ping-pong) unless that leaves SMs idle.
+  p.tiles = ((long long)((Nq + 255) / 256) * BH < num_sms()) ? 1 : 2;
+  p.nunits = (Nq + 128 * p.tiles - 1) / (128 * p.tiles);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal ? 1 : 0;
-  const long long blocks = (long long)p.npairs * BH;
+  const long long blocks = (long long)p.nunits * BH;
   if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   fa::fa_fwd_kernel<D><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -127,9 +157,9 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (Nk > 0) {
-    CUtensorMap mq, mk, mv, mdo;
+    CUtensorMap mq, mk, mv, mdo, mdq;
     if (!make_map_3d(&mq, q, D, Nq, BH) || !make_map_3d(&mk, k, D, Nk, BH) || !make_map_3d(&mv, v, D, Nk, BH) ||
-        !make_map_3d(&mdo, dO, D, Nq, BH))
+        !make_map_3d(&mdo, dO, D, Nq, BH) || !make_map_3d_f32(&mdq, dq_acc, D, Nq > 0 ? Nq : 1, BH))
       return FA_ERR_CUDA;
     if (!set_smem(fa::fa_bwd_main_kernel<D>, T::SMEM_BYTES)) return FA_ERR_CUDA;
     fa::BwdParams p;
@@ -147,7 +177,7 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.causal = causal ? 1 : 0;
     const long long blocks = (long long)p.nkt * BH;
     if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-    fa::fa_bwd_main_kernel<D><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, p);
+    fa::fa_bwd_main_kernel<D><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (rows > 0) {

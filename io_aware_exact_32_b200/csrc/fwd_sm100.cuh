@@ -78,16 +78,17 @@ struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
   int Nq, Nk, BH;
-  int npairs;        // ceil(Nq / 256)
+  int nunits;        // query units per (batch, head): ceil(Nq / (128 * tiles))
+  int tiles;         // 128-row query tiles per CTA: 2 (ping-pong), or 1 when the grid would be small
   float scale_log2;  // scale * log2(e)
   int causal;
 };
 
-// Number of 128-key tiles the CTA owning query rows [q0, q0 + 256) must visit.
-__device__ __forceinline__ int fwd_num_kv_tiles(int q0, int Nq, int Nk, int causal) {
+// Number of 128-key tiles the CTA owning query rows [q0, q0 + span) must visit.
+__device__ __forceinline__ int fwd_num_kv_tiles(int q0, int span, int Nq, int Nk, int causal) {
   const int nkt = (Nk + 127) / 128;
   if (!causal) return nkt;
-  const int last = min(q0 + 255, Nq - 1);
+  const int last = min(q0 + span - 1, Nq - 1);
   const int kmax = last + Nk - Nq;  // last visible key of the last row
   if (kmax < 0) return 1;           // every row fully masked: one tile, all -inf
   return min(nkt, kmax / 128 + 1);
@@ -154,9 +155,10 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.x % p.BH;
   const int rank = blockIdx.x / p.BH;
-  const int pair = p.causal ? (p.npairs - 1 - rank) : rank;  // causal: heaviest tiles first
-  const int q0 = pair * 256;
-  const int n_kv = fwd_num_kv_tiles(q0, p.Nq, p.Nk, p.causal);
+  const int unit = p.causal ? (p.nunits - 1 - rank) : rank;  // causal: heaviest tiles first
+  const bool two = p.tiles == 2;
+  const int q0 = unit * 128 * p.tiles;
+  const int n_kv = fwd_num_kv_tiles(q0, 128 * p.tiles, p.Nq, p.Nk, p.causal);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(T::BAR_Q), 1);
@@ -190,6 +192,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
   if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
     const int t = warp >> 2;
+    if (t == 1 && !two) goto teardown;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row in the tile == TMEM lane
     const int row = q0 + 128 * t + r;   // query index within the head
@@ -320,7 +323,25 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       const uint32_t tO[2] = {tmem_base + T::col_o(0), tmem_base + T::col_o(1)};
       bool ok = mbar_wait(bar(T::BAR_Q), 0, abort_flag);
       int v_prev = -1;
-      for (int j = 0; ok && j < n_kv; ++j) {
+      if (!two) {
+        // One query tile: S(j) then PV(j), each stage released after its only MMA group.
+        for (int j = 0; ok && j < n_kv; ++j) {
+          const int ik = 2 * j, iv = 2 * j + 1;
+          const int sk = ik % T::NS, sv = iv % T::NS;
+          if (!(ok = mbar_wait(bar(T::BAR_KV_FULL + sk), (ik / T::NS) & 1, abort_flag))) break;
+          tc_fence_after();
+          fwd_issue_qk<D>(tS[0], q_smem[0], sbase + T::OFF_KV + sk * T::TILE_BYTES);
+          mma_commit(bar(T::BAR_S_FULL + 0));
+          release(ik);
+          if (!(ok = mbar_wait(bar(T::BAR_KV_FULL + sv), (iv / T::NS) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(bar(T::BAR_P_READY + 0), j & 1, abort_flag))) break;
+          tc_fence_after();
+          fwd_issue_pv<D>(tO[0], tS[0], sbase + T::OFF_KV + sv * T::TILE_BYTES, j > 0);
+          mma_commit(bar(T::BAR_O_DONE + 0));
+          release(iv);
+        }
+      }
+      for (int j = 0; two && ok && j < n_kv; ++j) {
         const int ik = 2 * j, iv = 2 * j + 1;
         const int sk = ik % T::NS, sv = iv % T::NS;
         const uint32_t k_smem = sbase + T::OFF_KV + sk * T::TILE_BYTES;
@@ -346,7 +367,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
         mma_commit(bar(T::BAR_O_DONE + 0));
         v_prev = iv;
       }
-      if (ok && (ok = mbar_wait(bar(T::BAR_P_READY + 1), (n_kv - 1) & 1, abort_flag))) {
+      if (two && ok && (ok = mbar_wait(bar(T::BAR_P_READY + 1), (n_kv - 1) & 1, abort_flag))) {
         tc_fence_after();
         fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, n_kv - 1 > 0);
         mma_commit(bar(T::BAR_O_DONE + 1));
@@ -363,8 +384,8 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
   } else {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(T::BAR_Q), 2 * T::TILE_BYTES);
-      for (int t = 0; t < 2; ++t)
+      mbar_arrive_expect_tx(bar(T::BAR_Q), p.tiles * T::TILE_BYTES);
+      for (int t = 0; t < p.tiles; ++t)
         for (int b = 0; b < T::NBOX; ++b)
           tma_load_3d(sbase + T::OFF_Q + t * T::TILE_BYTES + b * T::BOX_BYTES, &tmQ, bar(T::BAR_Q), 64 * b,
                       q0 + 128 * t, bh);
@@ -393,6 +414,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
     __syncwarp();
   }
 
+teardown:
   tc_fence_before();
   __syncthreads();
   if (warp == 8) {
