@@ -56,7 +56,7 @@ struct BwdTraits {
   static constexpr int OFF_STAT = OFF_STG + STG_BYTES;         // [2][128] fp32: LSE*log2e, D
   static constexpr int OFF_BAR = OFF_STAT + 2 * 128 * 4;
   // barriers: kv_full | qd_full[NS] | qd_empty[NS] | s_full | ds_ready | ds_free | dq_full | dq_free |
-  //           acc_done | drain A | drain B
+  //           acc_done | drain A | drain B | sd_used | p_free
   static constexpr int BAR_KV = 0;
   static constexpr int BAR_QD_FULL = 1;
   static constexpr int BAR_QD_EMPTY = 1 + NS;
@@ -68,12 +68,18 @@ struct BwdTraits {
   static constexpr int BAR_ACC_DONE = BAR_S_FULL + 5;
   static constexpr int BAR_DRAIN = BAR_S_FULL + 6;
   static constexpr int BAR_DRAIN2 = BAR_S_FULL + 7;
-  static constexpr int NBAR = BAR_DRAIN2 + 1;
+  static constexpr int BAR_SD_USED = BAR_S_FULL + 8;  // S^T/dP^T of block i are in registers
+  static constexpr int BAR_P_FREE = BAR_S_FULL + 9;   // dV(i) has read P^T(i)
+  static constexpr int NBAR = BAR_P_FREE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   static constexpr uint32_t COL_DQ = SEP_DQ ? 256 + 2 * D : COL_DP;
+  // d = 64: P^T gets its own 64 columns, so the next block's S^T can be computed while this
+  // block's P^T still feeds dV.  d = 128: no room; P^T overwrites the first half of S^T.
+  static constexpr bool EARLY = SEP_DQ;
+  static constexpr uint32_t COL_P = EARLY ? 256 + 3 * D : COL_S;
   static constexpr int THREADS = 352;
   static constexpr uint32_t IDESC_SQ = make_idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
   static constexpr uint32_t IDESC_DVK = make_idesc_bf16(128, D, false, true);    // P^T dO, dS^T Q
@@ -201,6 +207,8 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     mbar_init(bar(T::BAR_ACC_DONE), 2);
     mbar_init(bar(T::BAR_DRAIN), 1);
     mbar_init(bar(T::BAR_DRAIN2), 1);
+    mbar_init(bar(T::BAR_SD_USED), 128);
+    mbar_init(bar(T::BAR_P_FREE), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -232,45 +240,75 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
       const int q0 = (i0 + it) * 128;
-      // Per-block statistics: LSE in log2 units (+inf past Nq) and D.  The first barrier keeps
-      // the previous block's readers ahead of the overwrite, the second publishes the new values.
-      float* st = stat;
+      // Per-block statistics, stored negated: -LSE in log2 units (-inf past Nq) and -D.  The
+      // first barrier keeps the previous block's readers ahead of the overwrite, the second
+      // publishes the new values.
       {
         const int q = q0 + r;
         const bool in = q < p.Nq;
         const size_t gi = (size_t)bh * p.Nq + (in ? q : 0);
-        const float lse2 = in ? p.lse[gi] * kLog2e : INFINITY;
-        const float dd = in ? p.dvec[gi] : 0.f;
+        const float nlse2 = in ? -p.lse[gi] * kLog2e : -INFINITY;
+        const float nd = in ? -p.dvec[gi] : 0.f;
         asm volatile("bar.sync 1, 128;" ::: "memory");
-        st[r] = lse2;
-        st[128 + r] = dd;
+        stat[r] = nlse2;
+        stat[128 + r] = nd;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
       ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL), it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       const int cmin = p.causal ? shift - q0 : -1;
+      // Masking is needed only where this warp holds a key past Nk or a causally hidden entry.
+      const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > 0);
+      const float4* st4 = reinterpret_cast<const float4*>(stat);
+      const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll 1
       for (int c32 = 0; c32 < 4; ++c32) {
         uint32_t sv[32], dpv[32];
         tmem_ld32x32b_x32_nowait(lane_addr + T::COL_S + 32 * c32, sv);
         tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DP + 32 * c32, dpv);
         tmem_wait_ld_2x32(sv, dpv);
+        if (T::EARLY && c32 == 3) {
+          // Both blocks of this iteration are now in registers: the issuers may overwrite them.
+          tc_fence_before();
+          mbar_arrive(bar(T::BAR_SD_USED));
+        }
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
+        for (int i = 0; i < 32; i += 4) {
           const int c = 32 * c32 + i;
-          const bool v0 = key_ok && (c >= cmin), v1 = key_ok && (c + 1 >= cmin);
-          const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sv[i]), p.scale_log2, -st[c])) : 0.f;
-          const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sv[i + 1]), p.scale_log2, -st[c + 1])) : 0.f;
-          const float d0 = p0 * (__uint_as_float(dpv[i]) - st[128 + c]);
-          const float d1 = p1 * (__uint_as_float(dpv[i + 1]) - st[128 + c + 1]);
-          pk[i / 2] = pack_bf16x2(p0, p1);
-          dk[i / 2] = pack_bf16x2(d0, d1);
+          const float4 nl = st4[c >> 2];        // broadcast: every lane reads the same address
+          const float4 nd = st4[32 + (c >> 2)];
+          const float2 x01 = ffma2(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), sc2,
+                                   make_float2(nl.x, nl.y));
+          const float2 x23 = ffma2(make_float2(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3])), sc2,
+                                   make_float2(nl.z, nl.w));
+          float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+          float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+          if (masked) {
+            p01.x = (key_ok && c >= cmin) ? p01.x : 0.f;
+            p01.y = (key_ok && c + 1 >= cmin) ? p01.y : 0.f;
+            p23.x = (key_ok && c + 2 >= cmin) ? p23.x : 0.f;
+            p23.y = (key_ok && c + 3 >= cmin) ? p23.y : 0.f;
+          }
+          const float2 t01 = fadd2(make_float2(__uint_as_float(dpv[i]), __uint_as_float(dpv[i + 1])),
+                                   make_float2(nd.x, nd.y));
+          const float2 t23 = fadd2(make_float2(__uint_as_float(dpv[i + 2]), __uint_as_float(dpv[i + 3])),
+                                   make_float2(nd.z, nd.w));
+          const float2 d01 = fmul2(p01, t01), d23 = fmul2(p23, t23);
+          pk[i / 2] = pack_bf16x2(p01.x, p01.y);
+          pk[i / 2 + 1] = pack_bf16x2(p23.x, p23.y);
+          dk[i / 2] = pack_bf16x2(d01.x, d01.y);
+          dk[i / 2 + 1] = pack_bf16x2(d23.x, d23.y);
         }
-        // P^T chunk -> TMEM (first 64 columns of the S^T block, bf16 pairs).  The S^T columns
-        // are free: S_FULL also covers issuer A's dV(it-1), the reader of P^T(it-1).
-        tmem_st32x32b_x16(lane_addr + T::COL_S + 16 * c32, pk);
+        // P^T chunk -> TMEM (bf16 pairs).  d = 128: over the consumed first half of S^T (S_FULL
+        // also covers issuer A's dV(it-1)); d = 64: into its own columns once dV(it-1) has read them.
+        if (T::EARLY && c32 == 0 && it > 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_P_FREE), (it - 1) & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        tmem_st32x32b_x16(lane_addr + T::COL_P + 16 * c32, pk);
         // dS^T(it-1) must have been read by dQ(it-1) and dK(it-1) before it is overwritten.
         if (c32 == 0 && it > 0) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DS_FREE), (it - 1) & 1, abort_flag));
@@ -409,17 +447,28 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       for (int it = 0; ok && it < n_q; ++it) {
         const uint32_t qs = q_smem(it), dos = qs + T::TILE_BYTES;
         const bool more = it + 1 < n_q;
+        if (T::EARLY && more) {
+          // d = 64: the next block's S^T / dP^T as soon as this block's are in registers.
+          if (!(ok = mbar_wait(bar(T::BAR_SD_USED), it & 1, abort_flag))) break;
+          if (!(ok = wait_qd(it + 1))) break;
+          tc_fence_after();
+          if (is_a) bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(it + 1));
+          else bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(it + 1) + T::TILE_BYTES);
+          mma_commit(bar(T::BAR_S_FULL));
+        }
         if (!(ok = mbar_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
         tc_fence_after();
         if (is_a) {
-          // dV_j += P^T dO_i  (P^T from TMEM, dO MN-major); then the next block's S^T, which
-          // overwrites P^T(it) only after dV(it) (same issuing thread, executed in order).
+          // dV_j += P^T dO_i  (P^T from TMEM, dO MN-major).
           const uint64_t do_mn = make_sdesc_sw128(dos, T::BOX_BYTES, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDV, tS + kk * 8, do_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK, (it > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tDV, tmem_base + T::COL_P + kk * 8, do_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          if (T::EARLY) mma_commit(bar(T::BAR_P_FREE));
           if (it + T::NS < n_q) mma_commit(bar(T::BAR_QD_EMPTY + it % T::NS));
-          if (more) {
+          if (!T::EARLY && more) {
+            // d = 128: the next S^T overwrites P^T(it) only after dV(it) (same thread, in order).
             if (!(ok = wait_qd(it + 1))) break;
             tc_fence_after();
             bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(it + 1));
@@ -434,10 +483,10 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
             mma_ss(tDQ, ds_mn + (uint64_t)((kk * 2048) >> 4), k_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DQ,
                    kk > 0 ? 1u : 0u);
           mma_commit(bar(T::BAR_DQ_FULL));
-          // Next block's dP^T (at d = 128 it reuses the dQ columns: wait until dQ(it) is read out).
-          if (more) {
+          // d = 128: the next block's dP^T reuses the dQ columns, once dQ(it) is read out.
+          if (!T::EARLY && more) {
             if (!(ok = wait_qd(it + 1))) break;
-            if (!T::SEP_DQ && !(ok = mbar_wait(bar(T::BAR_DQ_FREE), it & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(bar(T::BAR_DQ_FREE), it & 1, abort_flag))) break;
             tc_fence_after();
             bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(it + 1) + T::TILE_BYTES);
             mma_commit(bar(T::BAR_S_FULL));
