@@ -20,12 +20,13 @@
 //         dQ block reuses the dP^T columns once dP^T has been consumed)
 //   SMEM: K_j, V_j (resident), a ring of (Q_i, dO_i) stages, dS^T (bf16, 128-byte swizzle),
 //         and at d = 64 an fp32 staging tile for the dQ block
-//   warps 0-3: one thread per key row: P, dS (the critical path), dK/dV epilogue
-//   warps 4-7: one thread per query row of the dQ block: read it out of TMEM, release the
-//              columns at once, then add it into the fp32 accumulator (d = 64: one TMA bulk
+//   P/dS warpgroup(s): one thread per key row (d = 64: two groups, 64 query columns each):
+//              P, dS (the critical path), dK/dV epilogue
+//   dQ warpgroup: one thread per query row of the dQ block: read it out of TMEM, release the
+//              columns at once, then add it into the fp32 accumulator (d = 64: TMA bulk
 //              reduce-add of the staged tile; d = 128: per-thread atomics)
-//   warp 8: MMA issuer A (S^T, dV: the users of the S^T/P^T columns)
-//   warp 9: MMA issuer B (dP^T, dQ, dK); warp 10: TMA producer.
+//   MMA issuer A (S^T, dV: the users of the S^T/P^T columns), MMA issuer B (dP^T, dQ, dK),
+//   and a TMA producer warp.
 // Two issuers because one thread issues at most one 128 x N x 16 MMA every ~115 cycles
 // (measured on B200), about half the tensor-core rate at N = 128.  Each issuer runs one
 // iteration ahead: right after the MMAs that consume block i it issues the next block's S^T /
@@ -80,7 +81,14 @@ struct BwdTraits {
   // block's P^T still feeds dV.  d = 128: no room; P^T overwrites the first half of S^T.
   static constexpr bool EARLY = SEP_DQ;
   static constexpr uint32_t COL_P = EARLY ? 256 + 3 * D : COL_S;
-  static constexpr int THREADS = 352;
+  // P/dS warpgroups: at d = 64 two groups split the 128 query columns of every key row (the
+  // per-row chain of TMEM loads is the critical path); at d = 128 the registers of the dQ
+  // warpgroup's full rows leave no room for a second group.
+  static constexpr int NCWG = (D == 64) ? 2 : 1;
+  static constexpr int CW = 128 / NCWG;                 // query columns per P/dS warpgroup
+  static constexpr int WARP_DQ = 4 * NCWG;              // first warp of the dQ warpgroup
+  static constexpr int WARP_A = WARP_DQ + 4, WARP_B = WARP_DQ + 5, WARP_TMA = WARP_DQ + 6;
+  static constexpr int THREADS = 32 * (WARP_TMA + 1);
   static constexpr uint32_t IDESC_SQ = make_idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
   static constexpr uint32_t IDESC_DVK = make_idesc_bf16(128, D, false, true);    // P^T dO, dS^T Q
   static constexpr uint32_t IDESC_DQ = make_idesc_bf16(128, D, true, true);      // dS K
@@ -200,23 +208,23 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       mbar_init(bar(T::BAR_QD_EMPTY + s), 2);  // issuer A after dV, issuer B after dK
     }
     mbar_init(bar(T::BAR_S_FULL), 2);  // issuer A after S^T, issuer B after dP^T
-    mbar_init(bar(T::BAR_DS_READY), 128);
+    mbar_init(bar(T::BAR_DS_READY), 128 * T::NCWG);
     mbar_init(bar(T::BAR_DS_FREE), 1);  // issuer B after dQ and dK (the readers of dS^T)
     mbar_init(bar(T::BAR_DQ_FULL), 1);
     mbar_init(bar(T::BAR_DQ_FREE), 128);
     mbar_init(bar(T::BAR_ACC_DONE), 2);
     mbar_init(bar(T::BAR_DRAIN), 1);
     mbar_init(bar(T::BAR_DRAIN2), 1);
-    mbar_init(bar(T::BAR_SD_USED), 128);
+    mbar_init(bar(T::BAR_SD_USED), 128 * T::NCWG);
     mbar_init(bar(T::BAR_P_FREE), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == T::WARP_A) {
     tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 10 && lane == 0) {
+  if (warp == T::WARP_TMA && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -228,12 +236,14 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 4) {
-    // ------------------------------------------------------------------ P / dS warpgroup
-    const int r = warp * 32 + lane;  // key row in the block == TMEM lane
+  if (warp < T::WARP_DQ) {
+    // ------------------------------------------------------------------ P / dS warpgroup(s)
+    const int wg = warp >> 2;            // which column half (d = 64) or the only group (d = 128)
+    const int cb = wg * T::CW;           // first query column of this group
+    const int r = (warp & 3) * 32 + lane;  // key row in the block == TMEM lane
     const int key = k0 + r;
     const bool key_ok = key < p.Nk;
-    const uint32_t lane_addr = tmem_base + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_addr = tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
     // Query column c of block i sees this key iff c >= cmin (bottom-right causal alignment).
     const int shift = key - (p.Nk - p.Nq);
     const uint32_t ds_row = sbase + T::OFF_DS + r * 128;
@@ -249,40 +259,45 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
         const size_t gi = (size_t)bh * p.Nq + (in ? q : 0);
         const float nlse2 = in ? -p.lse[gi] * kLog2e : -INFINITY;
         const float nd = in ? -p.dvec[gi] : 0.f;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        stat[r] = nlse2;
-        stat[128 + r] = nd;
+        asm volatile("bar.sync 1, %0;" ::"n"(128 * T::NCWG) : "memory");
+        if (wg == 0) {
+          stat[r] = nlse2;
+          stat[128 + r] = nd;
+        }
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(128 * T::NCWG) : "memory");
       ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL), it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       const int cmin = p.causal ? shift - q0 : -1;
       // Masking is needed only where this warp holds a key past Nk or a causally hidden entry.
-      const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > 0);
+      const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > cb);
       const float4* st4 = reinterpret_cast<const float4*>(stat);
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-#pragma unroll 1
-      for (int c32 = 0; c32 < 4; ++c32) {
-        uint32_t sv[32], dpv[32];
-        tmem_ld32x32b_x32_nowait(lane_addr + T::COL_S + 32 * c32, sv);
-        tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DP + 32 * c32, dpv);
-        tmem_wait_ld_2x32(sv, dpv);
-        if (T::EARLY && c32 == 3) {
-          // Both blocks of this iteration are now in registers: the issuers may overwrite them.
-          tc_fence_before();
-          mbar_arrive(bar(T::BAR_SD_USED));
-        }
-        uint32_t pk[16], dk[16];
+      // 16-column chunks, double-buffered: the load of chunk c+1 is issued right after chunk c
+      // has arrived and overlaps its arithmetic (a TMEM load wait covers every load in flight).
+      constexpr int NCH = T::CW / 16;  // 16-column chunks of this group
+      uint32_t sv[2][16], dpv[2][16];
+      tmem_ld32x32b_x16_nowait(lane_addr + T::COL_S + cb, sv[0]);
+      tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb, dpv[0]);
+      tmem_wait_ld_2x16(sv[0], dpv[0]);
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const int c = 32 * c32 + i;
+      for (int ch = 0; ch < NCH; ++ch) {
+        const int cur = ch & 1;
+        if (ch < NCH - 1) {
+          tmem_ld32x32b_x16_nowait(lane_addr + T::COL_S + cb + 16 * (ch + 1), sv[cur ^ 1]);
+          tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb + 16 * (ch + 1), dpv[cur ^ 1]);
+        }
+        uint32_t pk[8], dk[8];
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const int c = cb + 16 * ch + i;
           const float4 nl = st4[c >> 2];        // broadcast: every lane reads the same address
           const float4 nd = st4[32 + (c >> 2)];
-          const float2 x01 = ffma2(make_float2(__uint_as_float(sv[i]), __uint_as_float(sv[i + 1])), sc2,
+          const float2 x01 = ffma2(make_float2(__uint_as_float(sv[cur][i]), __uint_as_float(sv[cur][i + 1])), sc2,
                                    make_float2(nl.x, nl.y));
-          const float2 x23 = ffma2(make_float2(__uint_as_float(sv[i + 2]), __uint_as_float(sv[i + 3])), sc2,
-                                   make_float2(nl.z, nl.w));
+          const float2 x23 = ffma2(make_float2(__uint_as_float(sv[cur][i + 2]), __uint_as_float(sv[cur][i + 3])),
+                                   sc2, make_float2(nl.z, nl.w));
           float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
           float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
           if (masked) {
@@ -291,9 +306,9 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
             p23.x = (key_ok && c + 2 >= cmin) ? p23.x : 0.f;
             p23.y = (key_ok && c + 3 >= cmin) ? p23.y : 0.f;
           }
-          const float2 t01 = fadd2(make_float2(__uint_as_float(dpv[i]), __uint_as_float(dpv[i + 1])),
+          const float2 t01 = fadd2(make_float2(__uint_as_float(dpv[cur][i]), __uint_as_float(dpv[cur][i + 1])),
                                    make_float2(nd.x, nd.y));
-          const float2 t23 = fadd2(make_float2(__uint_as_float(dpv[i + 2]), __uint_as_float(dpv[i + 3])),
+          const float2 t23 = fadd2(make_float2(__uint_as_float(dpv[cur][i + 2]), __uint_as_float(dpv[cur][i + 3])),
                                    make_float2(nd.z, nd.w));
           const float2 d01 = fmul2(p01, t01), d23 = fmul2(p23, t23);
           pk[i / 2] = pack_bf16x2(p01.x, p01.y);
@@ -301,27 +316,33 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           dk[i / 2] = pack_bf16x2(d01.x, d01.y);
           dk[i / 2 + 1] = pack_bf16x2(d23.x, d23.y);
         }
-        // P^T chunk -> TMEM (bf16 pairs).  d = 128: over the consumed first half of S^T (S_FULL
-        // also covers issuer A's dV(it-1)); d = 64: into its own columns once dV(it-1) has read them.
-        if (T::EARLY && c32 == 0 && it > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_P_FREE), (it - 1) & 1, abort_flag));
-          if (!ok) break;
+        if (ch == 0 && it > 0) {
+          // d = 64: P^T(it-1) must have been read by dV(it-1).  Both: dS^T(it-1) must have been
+          // read by dQ(it-1) and dK(it-1) before it is overwritten.
+          if (T::EARLY) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_P_FREE), (it - 1) & 1, abort_flag));
+          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DS_FREE), (it - 1) & 1, abort_flag));
           tc_fence_after();
         }
-        tmem_st32x32b_x16(lane_addr + T::COL_P + 16 * c32, pk);
-        // dS^T(it-1) must have been read by dQ(it-1) and dK(it-1) before it is overwritten.
-        if (c32 == 0 && it > 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DS_FREE), (it - 1) & 1, abort_flag));
-          if (!ok) break;
-        }
-        // dS^T chunk -> shared memory, K-major with 128-byte swizzle (box = 64 query columns).
+        // P^T chunk -> TMEM (bf16 pairs).  d = 128: over the consumed first half of S^T (S_FULL
+        // also covers issuer A's dV(it-1)); d = 64: into its own columns.
+        tmem_st32x32b_x8(lane_addr + T::COL_P + cb / 2 + 8 * ch, pk);
+        // dS^T chunk (16 query columns = two 16-byte chunks) -> shared memory, K-major with
+        // 128-byte swizzle (box = 64 query columns).
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int kc = 4 * c32 + m;  // 16-byte chunk index along the 128 query columns
+        for (int m = 0; m < 2; ++m) {
+          const int kc = cb / 8 + 2 * ch + m;  // 16-byte chunk index along the 128 query columns
           const uint32_t addr = ds_row + (kc >> 3) * T::BOX_BYTES + (((kc & 7) ^ (r & 7)) << 4);
           asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk[4 * m]), "r"(dk[4 * m + 1]),
                        "r"(dk[4 * m + 2]), "r"(dk[4 * m + 3])
                        : "memory");
+        }
+        if (ch < NCH - 1) {
+          tmem_wait_ld_2x16(sv[cur ^ 1], dpv[cur ^ 1]);
+          if (T::EARLY && ch == NCH - 2) {
+            // Both blocks of this iteration are now in registers: the issuers may overwrite them.
+            tc_fence_before();
+            mbar_arrive(bar(T::BAR_SD_USED));
+          }
         }
       }
       if (!ok) break;
@@ -330,9 +351,11 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       tc_fence_before();
       mbar_arrive(bar(T::BAR_DS_READY));
     }
-    // dK, dV epilogue.
-    if (ok && n_q > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_ACC_DONE), 0, abort_flag));
-    if (ok) {
+    // dK, dV epilogue (group 0 owns it; at d = 64 both groups hold the same key rows).
+    if (ok && wg == 0 && n_q > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_ACC_DONE), 0, abort_flag));
+    if (!ok) {
+      *abort_flag = 1;
+    } else if (wg == 0) {
       tc_fence_after();
       const size_t off = ((size_t)bh * p.Nk + (key_ok ? key : 0)) * D;
 #pragma unroll 1
@@ -359,15 +382,13 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           }
         }
       }
-    } else {
-      *abort_flag = 1;
     }
-  } else if (warp < 8) {
+  } else if (warp < T::WARP_DQ + 4) {
     // ------------------------------------------------------------------ dQ warpgroup
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // query row of the dQ block == TMEM lane
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    const bool leader = (warp == 4 && lane == 0);
+    const bool leader = (warp == T::WARP_DQ && lane == 0);
     const uint32_t stg_row = sbase + T::OFF_STG + r * 128;
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
@@ -425,9 +446,9 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     }
     if (!ok) *abort_flag = 1;
     if (T::SEP_DQ && leader) bulk_wait_group0();  // every reduce-add complete before the CTA exits
-  } else if (warp == 8 || warp == 9) {
+  } else if (warp == T::WARP_A || warp == T::WARP_B) {
     // ------------------------------------------------------------------ MMA issuers A and B
-    const bool is_a = (warp == 8);
+    const bool is_a = (warp == T::WARP_A);
     if (lane == 0 && n_q > 0) {
       const uint32_t k_smem = sbase + T::OFF_K, v_smem = sbase + T::OFF_V, ds_smem = sbase + T::OFF_DS;
       const uint32_t tS = tmem_base + T::COL_S, tDP = tmem_base + T::COL_DP, tDQ = tmem_base + T::COL_DQ;
@@ -546,7 +567,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == T::WARP_A) {
     tc_fence_after();
     tmem_dealloc(tmem_base, T::TMEM_COLS);
   }
