@@ -34,6 +34,8 @@
 // (S^T and dP^T ready, a Q/dO stage free, final dK/dV) count two commits.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100_ptx.cuh"
 
 namespace fa {
@@ -163,7 +165,7 @@ __device__ __forceinline__ void bwd_issue_ss_kmajor(uint32_t tmem_d, uint32_t a_
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint64_t off = (uint64_t)(((kk / 4) * T::BOX_BYTES + (kk % 4) * 32) >> 4);
-    mma_ss(tmem_d, ad + off, bd + off, T::IDESC_SQ, kk > 0 ? 1u : 0u);
+    mma_ss_w(tmem_d, ad + off, bd + off, T::IDESC_SQ, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -448,88 +450,94 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     if (T::SEP_DQ && leader) bulk_wait_group0();  // every reduce-add complete before the CTA exits
   } else if (warp == T::WARP_A || warp == T::WARP_B) {
     // ------------------------------------------------------------------ MMA issuers A and B
-    const bool is_a = (warp == T::WARP_A);
-    if (lane == 0 && n_q > 0) {
+    // Each issuer is a whole converged warp (one elected lane issues), and each runs its own
+    // specialised loop: no per-MMA branch on the issuer's role.
+    auto issuer = [&](auto role) {
+      constexpr bool is_a = decltype(role)::value;
       const uint32_t k_smem = sbase + T::OFF_K, v_smem = sbase + T::OFF_V, ds_smem = sbase + T::OFF_DS;
       const uint32_t tS = tmem_base + T::COL_S, tDP = tmem_base + T::COL_DP, tDQ = tmem_base + T::COL_DQ;
       const uint32_t tDV = tmem_base + T::COL_DV, tDK = tmem_base + T::COL_DK;
       auto q_smem = [&](int it) { return sbase + T::OFF_QD + (it % T::NS) * 2 * T::TILE_BYTES; };
-      auto wait_qd = [&](int it) { return mbar_wait(bar(T::BAR_QD_FULL + it % T::NS), (it / T::NS) & 1, abort_flag); };
+      auto wait_qd = [&](int it) { return warp_wait(bar(T::BAR_QD_FULL + it % T::NS), (it / T::NS) & 1, abort_flag); };
+      // The first operand block of this issuer's recomputed product: S^T = K Q^T (A) or dP^T = V dO^T (B).
+      auto issue_first = [&](int it) {
+        if constexpr (is_a) bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(it));
+        else bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(it) + T::TILE_BYTES);
+        mma_commit_w(bar(T::BAR_S_FULL));
+      };
       const uint64_t ds_kmaj = make_sdesc_sw128(ds_smem, 16, 1024);           // dS^T as A, K-major
       const uint64_t ds_mn = make_sdesc_sw128(ds_smem, T::BOX_BYTES, 1024);    // dS as A, MN-major
       const uint64_t k_mn = make_sdesc_sw128(k_smem, T::BOX_BYTES, 1024);      // K as B, MN-major
-      bool ok = mbar_wait(bar(T::BAR_KV), 0, abort_flag) && wait_qd(0);
+      bool ok = warp_wait(bar(T::BAR_KV), 0, abort_flag) && wait_qd(0);
       if (ok) {
         tc_fence_after();
-        if (is_a) bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(0));                   // S^T = K Q^T
-        else bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(0) + T::TILE_BYTES);       // dP^T = V dO^T
-        mma_commit(bar(T::BAR_S_FULL));
+        issue_first(0);
       }
       for (int it = 0; ok && it < n_q; ++it) {
         const uint32_t qs = q_smem(it), dos = qs + T::TILE_BYTES;
         const bool more = it + 1 < n_q;
         if (T::EARLY && more) {
           // d = 64: the next block's S^T / dP^T as soon as this block's are in registers.
-          if (!(ok = mbar_wait(bar(T::BAR_SD_USED), it & 1, abort_flag))) break;
+          if (!(ok = warp_wait(bar(T::BAR_SD_USED), it & 1, abort_flag))) break;
           if (!(ok = wait_qd(it + 1))) break;
           tc_fence_after();
-          if (is_a) bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(it + 1));
-          else bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(it + 1) + T::TILE_BYTES);
-          mma_commit(bar(T::BAR_S_FULL));
+          issue_first(it + 1);
         }
-        if (!(ok = mbar_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
+        if (!(ok = warp_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
         tc_fence_after();
-        if (is_a) {
+        if constexpr (is_a) {
           // dV_j += P^T dO_i  (P^T from TMEM, dO MN-major).
           const uint64_t do_mn = make_sdesc_sw128(dos, T::BOX_BYTES, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tDV, tmem_base + T::COL_P + kk * 8, do_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          if (T::EARLY) mma_commit(bar(T::BAR_P_FREE));
-          if (it + T::NS < n_q) mma_commit(bar(T::BAR_QD_EMPTY + it % T::NS));
+            mma_ts_w(tDV, tmem_base + T::COL_P + kk * 8, do_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK,
+                     (it > 0 || kk > 0) ? 1u : 0u);
+          if (T::EARLY) mma_commit_w(bar(T::BAR_P_FREE));
+          if (it + T::NS < n_q) mma_commit_w(bar(T::BAR_QD_EMPTY + it % T::NS));
           if (!T::EARLY && more) {
             // d = 128: the next S^T overwrites P^T(it) only after dV(it) (same thread, in order).
             if (!(ok = wait_qd(it + 1))) break;
             tc_fence_after();
-            bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(it + 1));
-            mma_commit(bar(T::BAR_S_FULL));
+            issue_first(it + 1);
           }
         } else {
           // dQ_i = dS K_j (A = dS, the MN-major view of dS^T), once the dQ columns are free.
-          if (T::SEP_DQ && it > 0 && !(ok = mbar_wait(bar(T::BAR_DQ_FREE), (it - 1) & 1, abort_flag))) break;
+          if (T::SEP_DQ && it > 0 && !(ok = warp_wait(bar(T::BAR_DQ_FREE), (it - 1) & 1, abort_flag))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDQ, ds_mn + (uint64_t)((kk * 2048) >> 4), k_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DQ,
-                   kk > 0 ? 1u : 0u);
-          mma_commit(bar(T::BAR_DQ_FULL));
+            mma_ss_w(tDQ, ds_mn + (uint64_t)((kk * 2048) >> 4), k_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DQ,
+                     kk > 0 ? 1u : 0u);
+          mma_commit_w(bar(T::BAR_DQ_FULL));
           // d = 128: the next block's dP^T reuses the dQ columns, once dQ(it) is read out.
           if (!T::EARLY && more) {
             if (!(ok = wait_qd(it + 1))) break;
-            if (!(ok = mbar_wait(bar(T::BAR_DQ_FREE), it & 1, abort_flag))) break;
+            if (!(ok = warp_wait(bar(T::BAR_DQ_FREE), it & 1, abort_flag))) break;
             tc_fence_after();
-            bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(it + 1) + T::TILE_BYTES);
-            mma_commit(bar(T::BAR_S_FULL));
+            issue_first(it + 1);
           }
           // dK_j += dS^T Q_i  (dS^T K-major, Q MN-major); scale is applied in the epilogue.
           const uint64_t q_mn = make_sdesc_sw128(qs, T::BOX_BYTES, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ss(tDK, ds_kmaj + (uint64_t)(((kk / 4) * T::BOX_BYTES + (kk % 4) * 32) >> 4),
-                   q_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK, (it > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar(T::BAR_DS_FREE));
-          if (it + T::NS < n_q) mma_commit(bar(T::BAR_QD_EMPTY + it % T::NS));
+            mma_ss_w(tDK, ds_kmaj + (uint64_t)(((kk / 4) * T::BOX_BYTES + (kk % 4) * 32) >> 4),
+                     q_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK, (it > 0 || kk > 0) ? 1u : 0u);
+          mma_commit_w(bar(T::BAR_DS_FREE));
+          if (it + T::NS < n_q) mma_commit_w(bar(T::BAR_QD_EMPTY + it % T::NS));
         }
       }
-      if (ok) mma_commit(bar(T::BAR_ACC_DONE));
+      if (ok) mma_commit_w(bar(T::BAR_ACC_DONE));
       if (!ok) {
         *abort_flag = 1;
         const int drain = is_a ? T::BAR_DRAIN : T::BAR_DRAIN2;
-        mma_commit(bar(drain));
+        mma_commit_w(bar(drain));
         const volatile int never = 0;
-        mbar_wait(bar(drain), 0, &never);
+        warp_wait(bar(drain), 0, &never);
       }
+    };
+    if (n_q > 0) {
+      if (warp == T::WARP_A) issuer(std::true_type{});
+      else issuer(std::false_type{});
     }
     __syncwarp();
   } else {

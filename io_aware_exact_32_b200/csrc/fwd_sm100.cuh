@@ -102,7 +102,7 @@ __device__ __forceinline__ void fwd_issue_qk(uint32_t tmem_d, uint32_t q_smem, u
   for (int kk = 0; kk < D / 16; ++kk) {
     // K advances 16 elements (32 bytes) inside a 128-byte swizzle row; every 4 steps, the next box.
     const uint64_t off = (uint64_t)(((kk / 4) * T::BOX_BYTES + (kk % 4) * 32) >> 4);
-    mma_ss(tmem_d, qd + off, kd + off, T::IDESC_QK, kk > 0 ? 1u : 0u);
+    mma_ss_w(tmem_d, qd + off, kd + off, T::IDESC_QK, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -113,7 +113,7 @@ __device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_d, uint32_t tmem_p, u
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk) {
     // 16 keys per step: P columns advance by 8 (two bf16 per 32-bit column), V rows by 16 x 128 B.
-    mma_ts(tmem_d, tmem_p + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), T::IDESC_PV,
+    mma_ts_w(tmem_d, tmem_p + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), T::IDESC_PV,
            (accumulate || kk > 0) ? 1u : 0u);
   }
 }
@@ -312,32 +312,32 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {  // the whole warp, converged: one elected lane issues
       const int total_loads = 2 * n_kv;
       auto release = [&](int load_idx) {
         // Only stages the producer will refill get an "empty" arrival.
-        if (load_idx + T::NS < total_loads) mma_commit(bar(T::BAR_KV_EMPTY + load_idx % T::NS));
+        if (load_idx + T::NS < total_loads) mma_commit_w(bar(T::BAR_KV_EMPTY + load_idx % T::NS));
       };
       const uint32_t q_smem[2] = {sbase + T::OFF_Q, sbase + T::OFF_Q + T::TILE_BYTES};
       const uint32_t tS[2] = {tmem_base + T::col_s(0), tmem_base + T::col_s(1)};
       const uint32_t tO[2] = {tmem_base + T::col_o(0), tmem_base + T::col_o(1)};
-      bool ok = mbar_wait(bar(T::BAR_Q), 0, abort_flag);
+      bool ok = warp_wait(bar(T::BAR_Q), 0, abort_flag);
       int v_prev = -1;
       if (!two) {
         // One query tile: S(j) then PV(j), each stage released after its only MMA group.
         for (int j = 0; ok && j < n_kv; ++j) {
           const int ik = 2 * j, iv = 2 * j + 1;
           const int sk = ik % T::NS, sv = iv % T::NS;
-          if (!(ok = mbar_wait(bar(T::BAR_KV_FULL + sk), (ik / T::NS) & 1, abort_flag))) break;
+          if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sk), (ik / T::NS) & 1, abort_flag))) break;
           tc_fence_after();
           fwd_issue_qk<D>(tS[0], q_smem[0], sbase + T::OFF_KV + sk * T::TILE_BYTES);
-          mma_commit(bar(T::BAR_S_FULL + 0));
+          mma_commit_w(bar(T::BAR_S_FULL + 0));
           release(ik);
-          if (!(ok = mbar_wait(bar(T::BAR_KV_FULL + sv), (iv / T::NS) & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(bar(T::BAR_P_READY + 0), j & 1, abort_flag))) break;
+          if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sv), (iv / T::NS) & 1, abort_flag))) break;
+          if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), j & 1, abort_flag))) break;
           tc_fence_after();
           fwd_issue_pv<D>(tO[0], tS[0], sbase + T::OFF_KV + sv * T::TILE_BYTES, j > 0);
-          mma_commit(bar(T::BAR_O_DONE + 0));
+          mma_commit_w(bar(T::BAR_O_DONE + 0));
           release(iv);
         }
       }
@@ -346,38 +346,38 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
         const int sk = ik % T::NS, sv = iv % T::NS;
         const uint32_t k_smem = sbase + T::OFF_KV + sk * T::TILE_BYTES;
         const uint32_t v_smem = sbase + T::OFF_KV + sv * T::TILE_BYTES;
-        if (!(ok = mbar_wait(bar(T::BAR_KV_FULL + sk), (ik / T::NS) & 1, abort_flag))) break;
+        if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sk), (ik / T::NS) & 1, abort_flag))) break;
         tc_fence_after();
         fwd_issue_qk<D>(tS[0], q_smem[0], k_smem);
-        mma_commit(bar(T::BAR_S_FULL + 0));
+        mma_commit_w(bar(T::BAR_S_FULL + 0));
         if (j > 0) {
-          if (!(ok = mbar_wait(bar(T::BAR_P_READY + 1), (j - 1) & 1, abort_flag))) break;
+          if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (j - 1) & 1, abort_flag))) break;
           tc_fence_after();
           fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, j - 1 > 0);
-          mma_commit(bar(T::BAR_O_DONE + 1));
+          mma_commit_w(bar(T::BAR_O_DONE + 1));
           release(v_prev);
         }
         fwd_issue_qk<D>(tS[1], q_smem[1], k_smem);
-        mma_commit(bar(T::BAR_S_FULL + 1));
+        mma_commit_w(bar(T::BAR_S_FULL + 1));
         release(ik);
-        if (!(ok = mbar_wait(bar(T::BAR_KV_FULL + sv), (iv / T::NS) & 1, abort_flag))) break;
-        if (!(ok = mbar_wait(bar(T::BAR_P_READY + 0), j & 1, abort_flag))) break;
+        if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sv), (iv / T::NS) & 1, abort_flag))) break;
+        if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), j & 1, abort_flag))) break;
         tc_fence_after();
         fwd_issue_pv<D>(tO[0], tS[0], v_smem, j > 0);
-        mma_commit(bar(T::BAR_O_DONE + 0));
+        mma_commit_w(bar(T::BAR_O_DONE + 0));
         v_prev = iv;
       }
-      if (two && ok && (ok = mbar_wait(bar(T::BAR_P_READY + 1), (n_kv - 1) & 1, abort_flag))) {
+      if (two && ok && (ok = warp_wait(bar(T::BAR_P_READY + 1), (n_kv - 1) & 1, abort_flag))) {
         tc_fence_after();
         fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, n_kv - 1 > 0);
-        mma_commit(bar(T::BAR_O_DONE + 1));
+        mma_commit_w(bar(T::BAR_O_DONE + 1));
       }
       if (!ok) {
         *abort_flag = 1;
         // Let every MMA already issued finish before the CTA releases its tensor memory.
-        mma_commit(bar(T::BAR_DRAIN));
+        mma_commit_w(bar(T::BAR_DRAIN));
         const volatile int never = 0;
-        mbar_wait(bar(T::BAR_DRAIN), 0, &never);
+        warp_wait(bar(T::BAR_DRAIN), 0, &never);
       }
     }
     __syncwarp();
