@@ -73,20 +73,25 @@ struct BwdTraits {
   static constexpr int BAR_DRAIN2 = BAR_S_FULL + 7;
   static constexpr int BAR_SD_USED = BAR_S_FULL + 8;  // S^T/dP^T of block i are in registers
   static constexpr int BAR_P_FREE = BAR_S_FULL + 9;   // dV(i) has read P^T(i)
-  static constexpr int NBAR = BAR_P_FREE + 1;
+  static constexpr int BAR_DO_FREE = BAR_S_FULL + 10; // dV(i) has read dO(i) (d = 128: staging)
+  static constexpr int NBAR = BAR_DO_FREE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   static constexpr uint32_t COL_DQ = SEP_DQ ? 256 + 2 * D : COL_DP;
-  // d = 64: P^T gets its own 64 columns, so the next block's S^T can be computed while this
-  // block's P^T still feeds dV.  d = 128: no room; P^T overwrites the first half of S^T.
+  // Two P/dS warpgroups split the 128 query columns of every key row (the per-row chain of TMEM
+  // loads and exponentials is the critical path); each writes its 64 columns of P^T (32 TMEM
+  // columns of bf16 pairs).  d = 64: P^T has its own 64 columns, so the next block's S^T can be
+  // computed while this block's P^T still feeds dV.  d = 128: no room; each group's P^T
+  // overwrites the start of its own, already read, half of S^T.
   static constexpr bool EARLY = SEP_DQ;
   static constexpr uint32_t COL_P = EARLY ? 256 + 3 * D : COL_S;
-  // P/dS warpgroups: at d = 64 two groups split the 128 query columns of every key row (the
-  // per-row chain of TMEM loads is the critical path); at d = 128 the registers of the dQ
-  // warpgroup's full rows leave no room for a second group.
-  static constexpr int NCWG = (D == 64) ? 2 : 1;
+  static constexpr uint32_t P_WG_STRIDE = EARLY ? 32 : 64;  // TMEM columns between the groups' P^T
+  static __host__ __device__ constexpr uint32_t p_col(int kk) {  // P^T columns of K-step kk (16 queries)
+    return COL_P + (uint32_t)(kk / 4) * P_WG_STRIDE + (uint32_t)(kk % 4) * 8;
+  }
+  static constexpr int NCWG = 2;
   static constexpr int CW = 128 / NCWG;                 // query columns per P/dS warpgroup
   static constexpr int WARP_DQ = 4 * NCWG;              // first warp of the dQ warpgroup
   static constexpr int WARP_A = WARP_DQ + 4, WARP_B = WARP_DQ + 5, WARP_TMA = WARP_DQ + 6;
@@ -207,7 +212,9 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     mbar_init(bar(T::BAR_KV), 1);
     for (int s = 0; s < T::NS; ++s) {
       mbar_init(bar(T::BAR_QD_FULL + s), 1);
-      mbar_init(bar(T::BAR_QD_EMPTY + s), 2);  // issuer A after dV, issuer B after dK
+      // issuer B after dK; issuer A after dV (d = 64) or the dQ warpgroup once its staging in the
+      // dO tile is read out (d = 128)
+      mbar_init(bar(T::BAR_QD_EMPTY + s), 2);
     }
     mbar_init(bar(T::BAR_S_FULL), 2);  // issuer A after S^T, issuer B after dP^T
     mbar_init(bar(T::BAR_DS_READY), 128 * T::NCWG);
@@ -219,6 +226,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     mbar_init(bar(T::BAR_DRAIN2), 1);
     mbar_init(bar(T::BAR_SD_USED), 128 * T::NCWG);
     mbar_init(bar(T::BAR_P_FREE), 1);
+    mbar_init(bar(T::BAR_DO_FREE), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -327,7 +335,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
         }
         // P^T chunk -> TMEM (bf16 pairs).  d = 128: over the consumed first half of S^T (S_FULL
         // also covers issuer A's dV(it-1)); d = 64: into its own columns.
-        tmem_st32x32b_x8(lane_addr + T::COL_P + cb / 2 + 8 * ch, pk);
+        tmem_st32x32b_x8(lane_addr + T::COL_P + wg * T::P_WG_STRIDE + 8 * ch, pk);
         // dS^T chunk (16 query columns = two 16-byte chunks) -> shared memory, K-major with
         // 128-byte swizzle (box = 64 query columns).
 #pragma unroll
@@ -398,18 +406,13 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DQ_FULL), it & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t v[D];
-      if constexpr (D == 128) {
-        tmem_ld32x32b_x128_nowait(lane_addr + T::COL_DQ, v);
-        tmem_wait_ld_x128(v);
-      } else {
+      if constexpr (T::SEP_DQ) {
+        uint32_t v[D];
         tmem_ld32x32b_x64_nowait(lane_addr + T::COL_DQ, v);
         tmem_wait_ld_x64(v);
-      }
-      // The dQ columns are free as soon as they are in registers.
-      tc_fence_before();
-      mbar_arrive(bar(T::BAR_DQ_FREE));
-      if constexpr (T::SEP_DQ) {
+        // The dQ columns are free as soon as they are in registers.
+        tc_fence_before();
+        mbar_arrive(bar(T::BAR_DQ_FREE));
         // Stage the scaled block as two 32-column fp32 boxes in the 128-byte-swizzle layout (row r
         // at r*128 bytes of each box, 16-byte chunk c at (c ^ r%8)*16: a quarter-warp hits
         // distinct banks), then bulk reduce-add both boxes.
@@ -434,20 +437,57 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           bulk_commit_group();
         }
       } else {
-        const int q = q0 + r;
-        if (q < p.Nq) {
-          float* dst = p.dq_acc + ((size_t)bh * p.Nq + q) * D;
+        // d = 128: no shared memory is left for a separate staging buffer.  The dO tile of this
+        // block's stage is free once dV(it) has read it; it takes the scaled dQ block in two
+        // 64-column halves (two 32-column fp32 boxes each), bulk reduce-added one after the other.
+        // The 128 TMEM columns are read as four 32-column chunks, two loads in flight, and are
+        // released once the last chunk is in registers.
+        const int s = it % T::NS;
+        const uint32_t stg = sbase + T::OFF_QD + s * 2 * T::TILE_BYTES + T::TILE_BYTES;
+        auto stage = [&](const uint32_t (&v)[32], int box) {
 #pragma unroll
-          for (int i = 0; i < D / 4; ++i) {
-            float4 a = make_float4(__uint_as_float(v[4 * i]) * p.scale, __uint_as_float(v[4 * i + 1]) * p.scale,
-                                   __uint_as_float(v[4 * i + 2]) * p.scale, __uint_as_float(v[4 * i + 3]) * p.scale);
-            atomicAdd(reinterpret_cast<float4*>(dst + 4 * i), a);
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t addr = stg + box * (128 * 128) + r * 128 + ((c ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                         "f"(__uint_as_float(v[4 * c]) * p.scale), "f"(__uint_as_float(v[4 * c + 1]) * p.scale),
+                         "f"(__uint_as_float(v[4 * c + 2]) * p.scale), "f"(__uint_as_float(v[4 * c + 3]) * p.scale)
+                         : "memory");
           }
-        }
+        };
+        auto reduce_half = [&](int h) {
+          fence_proxy_async_smem();
+          asm volatile("bar.sync 2, 128;" ::: "memory");
+          if (leader) {
+            // Rows past Nq fall outside the tensor map and are not written.
+            tma_reduce_add_3d(&tmDQ, stg, 64 * h, q0, bh);
+            tma_reduce_add_3d(&tmDQ, stg + 128 * 128, 64 * h + 32, q0, bh);
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the staging buffer is read out
+          }
+          asm volatile("bar.sync 2, 128;" ::: "memory");
+        };
+        uint32_t va[32], vb[32];
+        tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DQ, va);
+        tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DQ + 32, vb);
+        tmem_wait_ld_2x32(va, vb);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DO_FREE), it & 1, abort_flag));
+        if (!ok) break;
+        stage(va, 0);
+        stage(vb, 1);
+        tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DQ + 64, va);
+        tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DQ + 96, vb);
+        tmem_wait_ld_2x32(va, vb);
+        tc_fence_before();
+        mbar_arrive(bar(T::BAR_DQ_FREE));
+        reduce_half(0);
+        stage(va, 0);
+        stage(vb, 1);
+        reduce_half(1);
+        if (leader && it + T::NS < n_q) mbar_arrive(bar(T::BAR_QD_EMPTY + s));
       }
     }
     if (!ok) *abort_flag = 1;
-    if (T::SEP_DQ && leader) bulk_wait_group0();  // every reduce-add complete before the CTA exits
+    if (leader) bulk_wait_group0();  // every reduce-add complete before the CTA exits
   } else if (warp == T::WARP_A || warp == T::WARP_B) {
     // ------------------------------------------------------------------ MMA issuers A and B
     // Each issuer is a whole converged warp (one elected lane issues), and each runs its own
@@ -490,10 +530,15 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           const uint64_t do_mn = make_sdesc_sw128(dos, T::BOX_BYTES, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts_w(tDV, tmem_base + T::COL_P + kk * 8, do_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK,
+            mma_ts_w(tDV, tmem_base + T::p_col(kk), do_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK,
                      (it > 0 || kk > 0) ? 1u : 0u);
           if (T::EARLY) mma_commit_w(bar(T::BAR_P_FREE));
-          if (it + T::NS < n_q) mma_commit_w(bar(T::BAR_QD_EMPTY + it % T::NS));
+          if constexpr (T::SEP_DQ) {
+            if (it + T::NS < n_q) mma_commit_w(bar(T::BAR_QD_EMPTY + it % T::NS));
+          } else {
+            // d = 128: dO(it) becomes the dQ staging buffer; the dQ warpgroup frees the stage.
+            mma_commit_w(bar(T::BAR_DO_FREE));
+          }
           if (!T::EARLY && more) {
             // d = 128: the next S^T overwrites P^T(it) only after dV(it) (same thread, in order).
             if (!(ok = wait_qd(it + 1))) break;
