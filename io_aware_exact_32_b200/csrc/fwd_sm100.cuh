@@ -62,7 +62,8 @@ struct FwdTraits {
   static constexpr int BAR_P_READY = BAR_S_FULL + 2;
   static constexpr int BAR_O_DONE = BAR_P_READY + 2;
   static constexpr int BAR_DRAIN = BAR_O_DONE + 2;
-  static constexpr int NBAR = BAR_DRAIN + 1;
+  static constexpr int BAR_MERGE = BAR_DRAIN + 1;  // split mode: group 1's row statistics published
+  static constexpr int NBAR = BAR_MERGE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
@@ -79,7 +80,8 @@ struct FwdParams {
   float* lse;
   int Nq, Nk, BH;
   int nunits;        // query units per (batch, head): ceil(Nq / (128 * tiles))
-  int tiles;         // 128-row query tiles per CTA: 2 (ping-pong), or 1 when the grid would be small
+  int tiles;         // 128-row query tiles per CTA: 2 (ping-pong), or 1 when the grid would be small (then
+                     // the two softmax groups split that tile's key tiles: even / odd)
   float scale_log2;  // scale * log2(e)
   int causal;
 };
@@ -172,6 +174,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       mbar_init(bar(T::BAR_O_DONE + t), 1);
     }
     mbar_init(bar(T::BAR_DRAIN), 1);
+    mbar_init(bar(T::BAR_MERGE), 128);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -191,11 +194,13 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
 
   if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
+    // Two tiles: group t owns query tile t and visits every key tile.  Split (one query tile):
+    // group t visits key tiles t, t + 2, ... with its own running (m, l, O_t); group 0 merges.
     const int t = warp >> 2;
-    if (t == 1 && !two) goto teardown;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row in the tile == TMEM lane
-    const int row = q0 + 128 * t + r;   // query index within the head
+    const int row = q0 + (two ? 128 * t : 0) + r;  // query index within the head
+    const int n_own = two ? n_kv : (n_kv + 1 - t) / 2;  // key tiles this group visits
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
     const uint32_t colS = T::col_s(t), colO = T::col_o(t);
     int kmax = p.Nk - 1;  // last visible key of this row (inclusive)
@@ -203,8 +208,9 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
     float m_run = -INFINITY, l_run = 0.f, lr_run = 0.f;
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL + t), j & 1, abort_flag));
+    for (int step = 0; step < n_own; ++step) {
+      const int j = two ? step : 2 * step + t;  // key tile
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL + t), step & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
       // Load the S row in two halves; the second half's load overlaps the first half's max.
@@ -234,7 +240,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       bool resc = false;
       if (m_tile > m_run + kRescaleThreshold) {
         alpha = ex2_approx(m_run - m_tile);
-        resc = (j > 0) && (m_run != -INFINITY);
+        resc = (step > 0) && (m_run != -INFINITY);
         m_run = m_tile;
       }
       const float base = (m_run == -INFINITY) ? 0.f : m_run;
@@ -253,7 +259,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
         for (int c = 0; c < 16; ++c) {
           const float2 x = ffma2(make_float2(src[2 * c], src[2 * c + 1]), sc2, nb2);
           float2 e;
-          if (kPolyEvery > 0 && (c % kPolyEvery) == kPolyEvery - 1) {
+          if (kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
             e = exp2_poly2(x);
           } else {
             e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
@@ -269,8 +275,9 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       l_run = l_run * alpha + (tot_e.x + tot_e.y);
       lr_run = lr_run * alpha + (tot_r.x + tot_r.y);
       if (__any_sync(0xffffffffu, resc)) {
-        // O_t still holds the sum through tile j-1: wait until PV(j-1) has landed, then scale.
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (j - 1) & 1, abort_flag));
+        // O_t still holds the sum through this group's previous tile: wait until that PV has
+        // landed, then scale.
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (step - 1) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -286,8 +293,37 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       tc_fence_before();
       mbar_arrive(bar(T::BAR_P_READY + t));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (n_kv - 1) & 1, abort_flag));
-    if (ok) {
+    // This group's accumulator is complete once its last PV has landed.
+    if (ok && n_own > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (n_own - 1) & 1, abort_flag));
+    float* merge_stats = reinterpret_cast<float*>(smem + T::OFF_Q + T::TILE_BYTES);  // split: Q slot 1 unused
+    if (ok && !two && t == 1) {
+      // Split: publish (m, l, l of the rounded weights) for group 0, which merges both halves.
+      merge_stats[r] = m_run;
+      merge_stats[128 + r] = l_run;
+      merge_stats[256 + r] = lr_run;
+      mbar_arrive(bar(T::BAR_MERGE));
+    }
+    // Weights of O_0 and O_1 in the merged sum: the two-block identity of the online softmax (each
+    // group's sums are relative to its own running maximum).
+    float a0 = 1.f, a1 = 0.f;
+    bool use1 = false;
+    if (ok && !two && t == 0) {
+      // Split: group 1's statistics and (if it visited any key tile) its accumulator.
+      const int n1 = n_kv / 2;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_MERGE), 0, abort_flag));
+      if (ok && n1 > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + 1), (n1 - 1) & 1, abort_flag));
+      if (ok) {
+        const float m1 = merge_stats[r], l1 = merge_stats[128 + r], lr1 = merge_stats[256 + r];
+        const float m = fmaxf(m_run, m1);
+        a0 = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m);
+        a1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - m);
+        l_run = a0 * l_run + a1 * l1;
+        lr_run = a0 * lr_run + a1 * lr1;
+        m_run = m;
+        use1 = n1 > 0;
+      }
+    }
+    if (ok && (two || t == 0)) {
       tc_fence_after();
       const float inv = lr_run > 0.f ? 1.f / lr_run : 0.f;
       const bool in_range = row < p.Nq;
@@ -296,6 +332,16 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         tmem_ld32x32b_x32_wait(lane_addr + colO + 32 * c, o);
+        if (use1) {
+          uint32_t o1[32];
+          tmem_ld32x32b_x32_wait(lane_addr + T::col_o(1) + 32 * c, o1);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            o[i] = __float_as_uint(a0 * __uint_as_float(o[i]) + a1 * __uint_as_float(o1[i]));
+        } else if (!two) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(a0 * __uint_as_float(o[i]));
+        }
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -307,9 +353,8 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
         }
       }
       if (in_range) p.lse[(size_t)bh * p.Nq + row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
-    } else {
-      *abort_flag = 1;
     }
+    if (!ok) *abort_flag = 1;
   } else if (warp == 8) {
     // ------------------------------------------------------------------ MMA issuer
     {  // the whole warp, converged: one elected lane issues
@@ -324,21 +369,51 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       bool ok = warp_wait(bar(T::BAR_Q), 0, abort_flag);
       int v_prev = -1;
       if (!two) {
-        // One query tile: S(j) then PV(j), each stage released after its only MMA group.
-        for (int j = 0; ok && j < n_kv; ++j) {
-          const int ik = 2 * j, iv = 2 * j + 1;
-          const int sk = ik % T::NS, sv = iv % T::NS;
-          if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sk), (ik / T::NS) & 1, abort_flag))) break;
+        // Split: step i computes S_0 = Q K(2i)^T and S_1 = Q K(2i+1)^T, then O_0 += P_0 V(2i) and
+        // (one step later, like the two-tile order) O_1 += P_1 V(2i+1).  Loads arrive in the ring
+        // order K(j), V(j), K(j+1), V(j+1), ...
+        const int nsteps = (n_kv + 1) / 2;
+        int v1_prev = -1;  // load index of the V tile of group 1's pending PV
+        for (int i = 0; ok && i < nsteps; ++i) {
+          const int ik0 = 4 * i, iv0 = 4 * i + 1, ik1 = 4 * i + 2, iv1 = 4 * i + 3;
+          const bool has1 = 2 * i + 1 < n_kv;
+          if (!(ok = warp_wait(bar(T::BAR_KV_FULL + ik0 % T::NS), (ik0 / T::NS) & 1, abort_flag))) break;
           tc_fence_after();
-          fwd_issue_qk<D>(tS[0], q_smem[0], sbase + T::OFF_KV + sk * T::TILE_BYTES);
+          fwd_issue_qk<D>(tS[0], q_smem[0], sbase + T::OFF_KV + (ik0 % T::NS) * T::TILE_BYTES);
           mma_commit_w(bar(T::BAR_S_FULL + 0));
-          release(ik);
-          if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sv), (iv / T::NS) & 1, abort_flag))) break;
-          if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), j & 1, abort_flag))) break;
+          release(ik0);
+          if (v1_prev >= 0) {
+            if (!(ok = warp_wait(bar(T::BAR_KV_FULL + v1_prev % T::NS), (v1_prev / T::NS) & 1, abort_flag))) break;
+            if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (i - 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v1_prev % T::NS) * T::TILE_BYTES, i - 1 > 0);
+            mma_commit_w(bar(T::BAR_O_DONE + 1));
+            release(v1_prev);
+            v1_prev = -1;
+          }
+          if (has1) {
+            if (!(ok = warp_wait(bar(T::BAR_KV_FULL + ik1 % T::NS), (ik1 / T::NS) & 1, abort_flag))) break;
+            tc_fence_after();
+            fwd_issue_qk<D>(tS[1], q_smem[0], sbase + T::OFF_KV + (ik1 % T::NS) * T::TILE_BYTES);
+            mma_commit_w(bar(T::BAR_S_FULL + 1));
+            release(ik1);
+            v1_prev = iv1;
+          }
+          if (!(ok = warp_wait(bar(T::BAR_KV_FULL + iv0 % T::NS), (iv0 / T::NS) & 1, abort_flag))) break;
+          if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), i & 1, abort_flag))) break;
           tc_fence_after();
-          fwd_issue_pv<D>(tO[0], tS[0], sbase + T::OFF_KV + sv * T::TILE_BYTES, j > 0);
+          fwd_issue_pv<D>(tO[0], tS[0], sbase + T::OFF_KV + (iv0 % T::NS) * T::TILE_BYTES, i > 0);
           mma_commit_w(bar(T::BAR_O_DONE + 0));
-          release(iv);
+          release(iv0);
+        }
+        if (ok && v1_prev >= 0) {
+          const int i = nsteps - 1;
+          if ((ok = warp_wait(bar(T::BAR_KV_FULL + v1_prev % T::NS), (v1_prev / T::NS) & 1, abort_flag)) &&
+              (ok = warp_wait(bar(T::BAR_P_READY + 1), i & 1, abort_flag))) {
+            tc_fence_after();
+            fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v1_prev % T::NS) * T::TILE_BYTES, i > 0);
+            mma_commit_w(bar(T::BAR_O_DONE + 1));
+          }
         }
       }
       for (int j = 0; two && ok && j < n_kv; ++j) {
