@@ -405,15 +405,10 @@ def run_ours(args):
 
 
 def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
-    """d=128 causal N=4096 forward and forward+backward, and split-KV decode bandwidth."""
+    """d=128 causal forward and forward+backward at N = 4096, 8192, 16384 (the sweep's B*N = 16384
+    tokens, H=16), and split-KV decode bandwidth."""
     import torch
     res = {}
-    cfg = next(c for c in W.SWEEP if c.Nq == 4096 and c.d == 128)
-    x = W.make_config_inputs(cfg)
-    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
-    o, lse = fa.attention_forward(q, k, v, causal=True, scale=cfg.scale)
-    ws = torch.empty(fa.fa_bwd_workspace_size(cfg.B, cfg.H, cfg.Nq, cfg.d), dtype=torch.uint8, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
 
     def timed(fn):
         for _ in range(3):
@@ -429,16 +424,23 @@ def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
         torch.cuda.synchronize()
         return statistics.median(a.elapsed_time(b) for a, b in ts) / 1e3
 
-    t_f = timed(lambda: fa.fa_fwd(q, k, v, o, lse, True, cfg.scale, stream))
-    t_b = timed(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, True, cfg.scale, stream))
-    ff = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, True)
-    fb = W.flops_backward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, True)
-    res["causal_n4096_d128"] = {"fwd_tflops": ff / t_f / 1e12, "fwd_frac": ff / t_f / 1e12 / peaks["bf16_tflops"],
-                                "bwd_tflops": fb / t_b / 1e12,
-                                "fwd_bwd_tflops": (ff + fb) / (t_f + t_b) / 1e12,
-                                "fwd_bwd_frac": (ff + fb) / (t_f + t_b) / 1e12 / peaks["bf16_tflops"],
-                                "fwd_ms": 1e3 * t_f, "bwd_ms": 1e3 * t_b}
-    del q, k, v, do, o, lse, dq, dk, dv, ws
+    for n in (4096, 8192, 16384):
+        cfg = next(c for c in W.SWEEP if c.Nq == n and c.d == 128)
+        x = W.make_config_inputs(cfg)
+        q, k, v, do = (x[nm].to(dev) for nm in ("q", "k", "v", "do"))
+        o, lse = fa.attention_forward(q, k, v, causal=True, scale=cfg.scale)
+        ws = torch.empty(fa.fa_bwd_workspace_size(cfg.B, cfg.H, cfg.Nq, cfg.d), dtype=torch.uint8, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        t_f = timed(lambda: fa.fa_fwd(q, k, v, o, lse, True, cfg.scale, stream))
+        t_b = timed(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, True, cfg.scale, stream))
+        ff = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, True)
+        fb = W.flops_backward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, True)
+        fwd_t, fb_t = ff / t_f / 1e12, (ff + fb) / (t_f + t_b) / 1e12
+        res[f"causal_n{n}_d128"] = {"B": cfg.B, "H": cfg.H, "fwd_tflops": fwd_t, "fwd_frac": fwd_t / peaks["bf16_tflops"],
+                                    "fwd_frac_of_2250": fwd_t / 2250.0, "bwd_tflops": fb / t_b / 1e12,
+                                    "fwd_bwd_tflops": fb_t, "fwd_bwd_frac": fb_t / peaks["bf16_tflops"],
+                                    "fwd_bwd_frac_of_2250": fb_t / 2250.0, "fwd_ms": 1e3 * t_f, "bwd_ms": 1e3 * t_b}
+        del q, k, v, do, o, lse, dq, dk, dv, ws, x
     dc = W.DECODE
     xd = W.make_decode_inputs(dc.B, dc.H, dc.Lmax, dc.d, dc.lmin, dc.seed)
     qd, kc, vc = (xd[n].to(dev) for n in ("q", "k_cache", "v_cache"))

@@ -108,6 +108,7 @@ struct BwdParams {
   __nv_bfloat16* dk;  // [BH, Nk, D]
   __nv_bfloat16* dv;  // [BH, Nk, D]
   int Nq, Nk, BH, nkt;
+  int hgroup;         // heads per scheduling group (1 <= hgroup <= BH)
   float scale, scale_log2;
   int causal;
 };
@@ -174,17 +175,6 @@ __device__ __forceinline__ void bwd_issue_ss_kmajor(uint32_t tmem_d, uint32_t a_
   }
 }
 
-// TMA bulk reduce-add of a staged shared-memory tile into global memory (tensor map coordinates).
-__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
-  asm volatile("cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4}], [%1];"
-               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_group_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 template <int D>
 __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
@@ -201,8 +191,14 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
   float* stat = reinterpret_cast<float*>(smem + T::OFF_STAT);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x % p.BH;
-  const int jt = blockIdx.x / p.BH;
+  // Blocks run in groups of hgroup heads; inside a group, every key tile of those heads, the
+  // heaviest (causal) first.  The group's Q, dO and dQ accumulator then stay in L2 while its
+  // blocks sweep them, each block starting at its own query tile.
+  const int grp = blockIdx.x / (p.hgroup * p.nkt);
+  const int gsz = min(p.hgroup, p.BH - grp * p.hgroup);
+  const int r_in = blockIdx.x - grp * p.hgroup * p.nkt;
+  const int bh = grp * p.hgroup + r_in % gsz;
+  const int jt = r_in / gsz;
   const int k0 = jt * 128;
   const int nqt = (p.Nq + 127) / 128;
   const int i0 = bwd_first_q_tile(k0, p.Nq, p.Nk, p.causal);

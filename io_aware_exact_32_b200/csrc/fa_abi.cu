@@ -68,6 +68,19 @@ bool make_map_3d_f32(CUtensorMap* map, void* base, int D, int N, long long BH) {
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Multiprocessor count of the current device (cached per device).
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
 // Opt a kernel into its dynamic shared memory once per device.
 template <typename K>
 bool set_smem(K kernel, int bytes) {
@@ -83,19 +96,6 @@ bool set_smem(K kernel, int bytes) {
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
   if (ndone[dev] < 16) done[dev][ndone[dev]++] = reinterpret_cast<const void*>(kernel);
   return true;
-}
-
-// Multiprocessor count of the current device (cached per device).
-int num_sms() {
-  static int cache[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cache[dev] = n;
-  }
-  return cache[dev];
 }
 
 fa_status check_common(int B, int H, int Nq, int Nk, int d, float scale) {
@@ -172,6 +172,14 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.Nk = Nk;
     p.BH = BH;
     p.nkt = (Nk + 127) / 128;
+    // Heads per group: their Q and dO (bf16) and dQ accumulator (fp32), 8 Nq d bytes a head,
+    // within ~32 MB of the 126 MB L2; at least 4 heads so that a group fills the SMs.
+    {
+      const long long per_head = 8LL * Nq * D;
+      long long g = (32LL << 20) / (per_head > 0 ? per_head : 1);
+      g = g < 4 ? 4 : g;
+      p.hgroup = (int)(g < BH ? g : BH);
+    }
     p.scale = scale;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
