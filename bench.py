@@ -23,6 +23,7 @@ the max over ranks.  `--impl reference` times the float64 CPU oracle instead.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -77,6 +78,23 @@ def measured_peaks():
                 "source": "measured"}
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def captured_traffic(key):
+    """DRAM bytes per launch of a kernel, from the committed record of its ncu capture
+    (profiles/traffic.json), or (None, None) once the kernel's sources differ from the captured ones."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[key]
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["sources_sha256"]:
+            return None, None
+        return int(rec["dram_bytes_per_launch"]), rec["capture"]
+    except Exception:
+        return None, None
 
 
 class ClockSampler:
@@ -363,6 +381,11 @@ def run_ours(args):
                 "frac": dom_tflops / peaks["bf16_tflops"], "traffic": None,
                 "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
                 else "fallback 1590 TFLOP/s"}
+
+    if dom == "bwd":
+        roofline["traffic"], roofline["traffic_source"] = captured_traffic("fa_bwd_main_kernel<64> b2_h8_n1024_d64")
+        if roofline["traffic"] is not None:
+            roofline["traffic_unit"] = "bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)"
 
     extra = {}
     if not args.no_extra:
