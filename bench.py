@@ -463,6 +463,11 @@ def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
                                     "fwd_frac_of_2250": fwd_t / 2250.0, "bwd_tflops": fb / t_b / 1e12,
                                     "fwd_bwd_tflops": fb_t, "fwd_bwd_frac": fb_t / peaks["bf16_tflops"],
                                     "fwd_bwd_frac_of_2250": fb_t / 2250.0, "fwd_ms": 1e3 * t_f, "bwd_ms": 1e3 * t_b}
+        if n == 4096:
+            t_bd = timed(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, True, cfg.scale, stream,
+                                           deterministic=True))
+            res["deterministic_bwd_causal_n4096_d128"] = {"bwd_tflops": fb / t_bd / 1e12, "bwd_ms": 1e3 * t_bd,
+                                                          "vs_default_bwd": t_b / t_bd}
         del q, k, v, do, o, lse, dq, dk, dv, ws, x
     dc = W.DECODE
     xd = W.make_decode_inputs(dc.B, dc.H, dc.Lmax, dc.d, dc.lmin, dc.seed)

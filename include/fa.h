@@ -114,6 +114,24 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  void* stream);
 
 /*
+ * Deterministic backward: the same results as fa_bwd (same arguments, same
+ * workspace size query), with dQ bitwise reproducible run to run.
+ *
+ * dK and dV come from the key-block schedule of fa_bwd without its dQ part;
+ * dQ comes from a second pass with the query block stationary, which
+ * recomputes S and dP for each (query block, key block) pair and accumulates
+ * dQ_i = scale * sum_j dS_ij K_j on chip, so no two blocks add into the same dQ
+ * row (the nondeterminism of fa_bwd comes from the order of those adds,
+ * "Transformer、注意力机制与优化", section 为什么前向传播和反向传播的并行化策略不同).
+ * Costs two extra matrix products per pair (about 40% more tensor work).
+ */
+FA_API fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                 const void* dO, const float* lse, void* dq, void* dk, void* dv,
+                 void* workspace, size_t ws_bytes,
+                 int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                 void* stream);
+
+/*
  * Bytes of workspace fa_decode_splitkv needs for the per-split partial
  * results (m, l, unnormalised O) at the given split count (0 = the automatic
  * choice for this Lmax).  Returns 0 on invalid sizes.

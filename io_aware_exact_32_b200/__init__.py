@@ -6,7 +6,7 @@ dtypes and devices, passes raw device pointers and the current CUDA stream,
 and raises on a non-zero status.  PyTorch provides device memory and streams.
 
 C-ABI mirrors (same names, torch tensors in place of pointers):
-    fa_fwd, fa_bwd, fa_bwd_workspace_size, fa_decode_splitkv,
+    fa_fwd, fa_bwd, fa_bwd_deterministic, fa_bwd_workspace_size, fa_decode_splitkv,
     fa_decode_workspace_size, fa_decode_splitkv_noalloc, fa_get_device_error,
     fa_status_string, fa_version
 Convenience wrappers that allocate outputs:
@@ -20,7 +20,8 @@ import os
 
 __all__ = [
     "FAError", "lib", "lib_path",
-    "fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_decode_splitkv", "fa_decode_workspace_size",
+    "fa_fwd", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size", "fa_decode_splitkv",
+    "fa_decode_workspace_size",
     "fa_decode_splitkv_noalloc", "fa_get_device_error", "fa_status_string", "fa_version",
     "attention_forward", "attention_backward", "decode_splitkv",
 ]
@@ -57,6 +58,8 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_workspace_size.restype = sz
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, vp]
     L.fa_bwd.restype = i
+    L.fa_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, vp]
+    L.fa_bwd_deterministic.restype = i
     L.fa_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.fa_decode_workspace_size.restype = sz
     L.fa_decode_splitkv.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, f, i, vp, sz, vp]
@@ -135,8 +138,10 @@ def fa_bwd_workspace_size(B: int, H: int, Nq: int, d: int) -> int:
     return int(lib().fa_bwd_workspace_size(B, H, Nq, d))
 
 
-def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal: bool, scale=None, stream=None) -> None:
-    """dQ, dK, dV by recomputation (see include/fa.h: fa_bwd).  workspace: uint8 device tensor."""
+def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal: bool, scale=None, stream=None,
+           deterministic: bool = False) -> None:
+    """dQ, dK, dV by recomputation (see include/fa.h: fa_bwd, and fa_bwd_deterministic when
+    deterministic is set).  workspace: uint8 device tensor."""
     import torch
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
@@ -147,9 +152,15 @@ def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal: bool, scale=None,
         _need(t, n, torch.bfloat16, dev, shp)
     _need(lse, "lse", torch.float32, dev, (B, H, Nq))
     _need(workspace, "workspace", torch.uint8, dev)
-    _check(lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
-                        _ptr(workspace), workspace.numel(), B, H, Nq, Nk, d, _scale(scale, d),
-                        int(bool(causal)), _stream_ptr(stream)), "fa_bwd")
+    fn, name = (lib().fa_bwd_deterministic, "fa_bwd_deterministic") if deterministic else (lib().fa_bwd, "fa_bwd")
+    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+              _ptr(workspace), workspace.numel(), B, H, Nq, Nk, d, _scale(scale, d),
+              int(bool(causal)), _stream_ptr(stream)), name)
+
+
+def fa_bwd_deterministic(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal: bool, scale=None, stream=None) -> None:
+    """fa_bwd with bitwise reproducible dQ (see include/fa.h: fa_bwd_deterministic)."""
+    fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal, scale, stream, deterministic=True)
 
 
 def fa_decode_workspace_size(B: int, H: int, Lmax: int, d: int, num_splits: int = 0) -> int:
@@ -223,8 +234,10 @@ def attention_forward(q, k, v, causal: bool = False, scale=None, stream=None):
     return o, lse
 
 
-def attention_backward(q, k, v, o, lse, dO, causal: bool = False, scale=None, stream=None, workspace=None):
-    """Allocate dQ, dK, dV (and the workspace unless given) and run fa_bwd; returns (dq, dk, dv)."""
+def attention_backward(q, k, v, o, lse, dO, causal: bool = False, scale=None, stream=None, workspace=None,
+                       deterministic: bool = False):
+    """Allocate dQ, dK, dV (and the workspace unless given) and run fa_bwd (fa_bwd_deterministic when
+    deterministic is set); returns (dq, dk, dv)."""
     import torch
     B, H, Nq, d = q.shape
     dq = torch.empty_like(q)
@@ -232,7 +245,7 @@ def attention_backward(q, k, v, o, lse, dO, causal: bool = False, scale=None, st
     dv = torch.empty_like(v)
     if workspace is None:
         workspace = _workspace(fa_bwd_workspace_size(B, H, Nq, d), q.device)
-    fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal, scale, stream)
+    fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal, scale, stream, deterministic=deterministic)
     return dq, dk, dv
 
 

@@ -141,9 +141,11 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const __nv_bfloa
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (lane == 0) dvec[row] = acc;
-  float* qrow = dq_acc + row * D + lane * PER;
+  if (dq_acc) {  // null in the deterministic backward, which has no accumulator
+    float* qrow = dq_acc + row * D + lane * PER;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) qrow[i] = 0.f;
+    for (int i = 0; i < PER; ++i) qrow[i] = 0.f;
+  }
 }
 
 // dQ accumulator (already scaled) -> bf16, 8 elements per thread.
@@ -176,7 +178,8 @@ __device__ __forceinline__ void bwd_issue_ss_kmajor(uint32_t tmem_d, uint32_t a_
 }
 
 
-template <int D>
+// DQ = false (the deterministic backward): dK and dV only; dQ comes from fa_bwd_dq_kernel.
+template <int D, bool DQ = true>
 __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -397,7 +400,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     const bool leader = (warp == T::WARP_DQ && lane == 0);
     const uint32_t stg_row = sbase + T::OFF_STG + r * 128;
     bool ok = true;
-    for (int it = 0; it < n_q; ++it) {
+    for (int it = 0; it < (DQ ? n_q : 0); ++it) {
       const int q0 = (i0 + it) * 128;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DQ_FULL), it & 1, abort_flag));
       if (!ok) break;
@@ -529,7 +532,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
             mma_ts_w(tDV, tmem_base + T::p_col(kk), do_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DVK,
                      (it > 0 || kk > 0) ? 1u : 0u);
           if (T::EARLY) mma_commit_w(bar(T::BAR_P_FREE));
-          if constexpr (T::SEP_DQ) {
+          if constexpr (T::SEP_DQ || !DQ) {
             if (it + T::NS < n_q) mma_commit_w(bar(T::BAR_QD_EMPTY + it % T::NS));
           } else {
             // d = 128: dO(it) becomes the dQ staging buffer; the dQ warpgroup frees the stage.
@@ -542,18 +545,20 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
             issue_first(it + 1);
           }
         } else {
-          // dQ_i = dS K_j (A = dS, the MN-major view of dS^T), once the dQ columns are free.
-          if (T::SEP_DQ && it > 0 && !(ok = warp_wait(bar(T::BAR_DQ_FREE), (it - 1) & 1, abort_flag))) break;
-          tc_fence_after();
+          if constexpr (DQ) {
+            // dQ_i = dS K_j (A = dS, the MN-major view of dS^T), once the dQ columns are free.
+            if (T::SEP_DQ && it > 0 && !(ok = warp_wait(bar(T::BAR_DQ_FREE), (it - 1) & 1, abort_flag))) break;
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss_w(tDQ, ds_mn + (uint64_t)((kk * 2048) >> 4), k_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DQ,
-                     kk > 0 ? 1u : 0u);
-          mma_commit_w(bar(T::BAR_DQ_FULL));
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ss_w(tDQ, ds_mn + (uint64_t)((kk * 2048) >> 4), k_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DQ,
+                       kk > 0 ? 1u : 0u);
+            mma_commit_w(bar(T::BAR_DQ_FULL));
+          }
           // d = 128: the next block's dP^T reuses the dQ columns, once dQ(it) is read out.
           if (!T::EARLY && more) {
             if (!(ok = wait_qd(it + 1))) break;
-            if (!(ok = warp_wait(bar(T::BAR_DQ_FREE), it & 1, abort_flag))) break;
+            if (DQ && !(ok = warp_wait(bar(T::BAR_DQ_FREE), it & 1, abort_flag))) break;
             tc_fence_after();
             issue_first(it + 1);
           }

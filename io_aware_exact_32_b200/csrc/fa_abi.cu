@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/fa.h"
+#include "bwd_dq_sm100.cuh"
 #include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
@@ -143,17 +144,22 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// deterministic: dK/dV from the key-block kernel without its dQ part, and dQ from the
+// query-block kernel (no accumulator, no atomics).  With no key at all the regular path runs
+// (it only writes zeros).
 template <int D>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                      void* dq, void* dk, void* dv, void* ws, int BH, int Nq, int Nk, float scale, int causal,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, bool deterministic) {
+  if (Nk == 0) deterministic = false;
   using T = fa::BwdTraits<D>;
   const long long rows = (long long)BH * Nq;
   float* dvec = static_cast<float*>(ws);
   float* dq_acc = reinterpret_cast<float*>(static_cast<char*>(ws) + align256((size_t)rows * 4));
   if (rows > 0) {
     fa::fa_bwd_preprocess_kernel<D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), dvec, dq_acc, rows);
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), dvec,
+        deterministic ? nullptr : dq_acc, rows);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   }
   if (Nk > 0) {
@@ -161,7 +167,9 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     if (!make_map_3d(&mq, q, D, Nq, BH) || !make_map_3d(&mk, k, D, Nk, BH) || !make_map_3d(&mv, v, D, Nk, BH) ||
         !make_map_3d(&mdo, dO, D, Nq, BH) || !make_map_3d_f32(&mdq, dq_acc, D, Nq > 0 ? Nq : 1, BH))
       return FA_ERR_CUDA;
-    if (!set_smem(fa::fa_bwd_main_kernel<D>, T::SMEM_BYTES)) return FA_ERR_CUDA;
+    if (!set_smem(fa::fa_bwd_main_kernel<D, true>, T::SMEM_BYTES) ||
+        !set_smem(fa::fa_bwd_main_kernel<D, false>, T::SMEM_BYTES))
+      return FA_ERR_CUDA;
     fa::BwdParams p;
     p.lse = lse;
     p.dvec = dvec;
@@ -185,10 +193,32 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.causal = causal ? 1 : 0;
     const long long blocks = (long long)p.nkt * BH;
     if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-    fa::fa_bwd_main_kernel<D><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
+    if (deterministic)
+      fa::fa_bwd_main_kernel<D, false><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
+    else
+      fa::fa_bwd_main_kernel<D, true><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    if (deterministic && Nq > 0) {
+      using TQ = fa::DqTraits<D>;
+      if (!set_smem(fa::fa_bwd_dq_kernel<D>, TQ::SMEM_BYTES)) return FA_ERR_CUDA;
+      fa::DqParams pq;
+      pq.dq = static_cast<__nv_bfloat16*>(dq);
+      pq.lse = lse;
+      pq.dvec = dvec;
+      pq.Nq = Nq;
+      pq.Nk = Nk;
+      pq.BH = BH;
+      pq.nqt = (Nq + 127) / 128;
+      pq.scale = scale;
+      pq.scale_log2 = scale * 1.4426950408889634f;
+      pq.causal = causal ? 1 : 0;
+      const long long qblocks = (long long)pq.nqt * BH;
+      if (qblocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+      fa::fa_bwd_dq_kernel<D><<<(unsigned)qblocks, TQ::THREADS, TQ::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, pq);
+      if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
   }
-  if (rows > 0) {
+  if (rows > 0 && !deterministic) {
     const long long n8 = rows * D / 8;
     fa::fa_bwd_dq_convert_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, stream>>>(
         dq_acc, static_cast<__nv_bfloat16*>(dq), n8);
@@ -254,9 +284,9 @@ size_t fa_bwd_workspace_size(int B, int H, int Nq, int d) {
   return align256(rows * 4) + align256(rows * d * 4);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+static fa_status bwd_entry(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int Nq, int Nk, int d,
-                 float scale, int causal, void* stream) {
+                 float scale, int causal, void* stream, bool deterministic) {
   fa_status st = check_common(B, H, Nq, Nk, d, scale);
   if (st != FA_OK) return st;
   const long long BH = (long long)B * H;
@@ -271,8 +301,23 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (need > 0 && (!workspace || ws_bytes < need)) return FA_ERR_WORKSPACE;
   if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s)
-                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s);
+  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s, deterministic)
+                 : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s,
+                                   deterministic);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int Nq, int Nk, int d,
+                 float scale, int causal, void* stream) {
+  return bwd_entry(q, k, v, o, dO, lse, dq, dk, dv, workspace, ws_bytes, B, H, Nq, Nk, d, scale, causal, stream,
+                   false);
+}
+
+fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                               const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
+                               int H, int Nq, int Nk, int d, float scale, int causal, void* stream) {
+  return bwd_entry(q, k, v, o, dO, lse, dq, dk, dv, workspace, ws_bytes, B, H, Nq, Nk, d, scale, causal, stream,
+                   true);
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Lmax, int d, int num_splits) {
