@@ -96,9 +96,10 @@ FA_API size_t fa_bwd_workspace_size(int B, int H, int Nq, int d);
  * row-softmax gradient dS, dQ = dS K, dK = dS^T Q), with D_i = rowsum(dO_i * O_i)
  * and P recomputed from LSE alone ("FlashAttention 系列技术详解", section
  * 具体优化策略), and the column-block parallel schedule whose dQ partial sums
- * meet through atomic adds in device memory ("Transformer、注意力机制与优化",
- * section 为什么前向传播和反向传播的并行化策略不同).  dQ is therefore not
- * bitwise deterministic run to run.
+ * meet through reduce-adds in device memory ("Transformer、注意力机制与优化",
+ * section 为什么前向传播和反向传播的并行化策略不同; here TMA bulk reduce-adds of
+ * shared-memory-staged blocks).  The order of those adds varies, so dQ is not
+ * bitwise deterministic run to run (see fa_bwd_deterministic).
  *
  *   q, o, dO [B, H, Nq, d] bf16, read;  k, v [B, H, Nk, d] bf16, read
  *   lse      [B, H, Nq] fp32, read (as written by fa_fwd)
@@ -168,6 +169,36 @@ FA_API fa_status fa_decode_splitkv(const void* q, const void* k_cache, const voi
  * fa_decode_splitkv_noalloc.
  */
 #define FA_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * Sequence-parallel decode building blocks (several devices each hold a slice
+ * of every sequence's KV cache): the per-split partial results of
+ * fa_decode_splitkv, unmerged, and their merge.  The merge is the same
+ * (m, l, O) recurrence that combines splits on one device ("Transformer、注意力
+ * 机制与优化", section Flash-Decoding), so partials from several devices,
+ * gathered in one buffer, merge exactly like partials from one device.
+ *
+ * fa_decode_num_splits: the split count S fa_decode_partials uses for this
+ * Lmax and num_splits (0 on invalid arguments).
+ *
+ * fa_decode_partials: as fa_decode_splitkv for k_cache, v_cache [B, H, Lmax, d]
+ * and seqlens (device int32 [B], 0 <= L_b <= Lmax; a slice may be empty), but
+ * writes, for every (b, h) and split s, the unnormalised output
+ * part_o [B, H, S, d] fp32 and part_ml [B, H, S, 2] fp32 = (running max m in
+ * log2 units of scale * q.k, sum l of 2^(x - m)); an empty split gives
+ * (m, l) = (-inf, 0).  Buffers caller-owned, 16-byte aligned.
+ *
+ * fa_decode_merge: merges R groups of S partials (group r at offset r*B*H*S
+ * rows: the layout of an all-gather of per-device partials along the first
+ * dimension) into o [B, H, 1, d] bf16 and, if lse is not NULL, lse [B, H]
+ * fp32.  A (b, h) with no key at all gets o = 0 and lse = -inf.
+ */
+FA_API int fa_decode_num_splits(int Lmax, int num_splits);
+FA_API fa_status fa_decode_partials(const void* q, const void* k_cache, const void* v_cache,
+                                    const int* seqlens, int Lmax, float* part_o, float* part_ml,
+                                    int B, int H, int d, float scale, int num_splits, void* stream);
+FA_API fa_status fa_decode_merge(const float* part_o, const float* part_ml, int R, int S,
+                                 void* o, float* lse, int B, int H, int d, void* stream);
 
 /*
  * Split-KV decode that allocates nothing and takes no workspace.

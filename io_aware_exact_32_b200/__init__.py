@@ -6,7 +6,8 @@ dtypes and devices, passes raw device pointers and the current CUDA stream,
 and raises on a non-zero status.  PyTorch provides device memory and streams.
 
 C-ABI mirrors (same names, torch tensors in place of pointers):
-    fa_fwd, fa_bwd, fa_bwd_deterministic, fa_bwd_workspace_size, fa_decode_splitkv,
+    fa_fwd, fa_bwd, fa_bwd_deterministic, fa_bwd_workspace_size, fa_decode_splitkv, fa_decode_num_splits,
+    fa_decode_partials, fa_decode_merge,
     fa_decode_workspace_size, fa_decode_splitkv_noalloc, fa_get_device_error,
     fa_status_string, fa_version
 Convenience wrappers that allocate outputs:
@@ -21,7 +22,7 @@ import os
 __all__ = [
     "FAError", "lib", "lib_path",
     "fa_fwd", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size", "fa_decode_splitkv",
-    "fa_decode_workspace_size",
+    "fa_decode_workspace_size", "fa_decode_num_splits", "fa_decode_partials", "fa_decode_merge",
     "fa_decode_splitkv_noalloc", "fa_get_device_error", "fa_status_string", "fa_version",
     "attention_forward", "attention_backward", "decode_splitkv",
 ]
@@ -66,6 +67,12 @@ def lib() -> ctypes.CDLL:
     L.fa_decode_splitkv.restype = i
     L.fa_decode_splitkv_noalloc.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, f, i, vp]
     L.fa_decode_splitkv_noalloc.restype = i
+    L.fa_decode_num_splits.argtypes = [i, i]
+    L.fa_decode_num_splits.restype = i
+    L.fa_decode_partials.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, f, i, vp]
+    L.fa_decode_partials.restype = i
+    L.fa_decode_merge.argtypes = [vp, vp, i, i, vp, vp, i, i, i, vp]
+    L.fa_decode_merge.restype = i
     L.fa_get_device_error.argtypes = [vp]
     L.fa_get_device_error.restype = i
     L.fa_status_string.argtypes = [i]
@@ -212,6 +219,47 @@ def fa_decode_splitkv_noalloc(q, k_cache, v_cache, seqlens, o, lse, scale=None, 
     _check(lib().fa_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(o),
                                            _ptr(lse), B, H, d, _scale(scale, d), int(num_splits),
                                            _stream_ptr(stream)), "fa_decode_splitkv_noalloc")
+
+
+def fa_decode_num_splits(Lmax: int, num_splits: int = 0) -> int:
+    return int(lib().fa_decode_num_splits(Lmax, num_splits))
+
+
+def fa_decode_partials(q, k_cache, v_cache, seqlens, part_o, part_ml, scale=None, num_splits: int = 0,
+                       stream=None) -> None:
+    """Unmerged split-KV partials for a KV slice (see include/fa.h: fa_decode_partials).
+    part_o [B, H, S, d] fp32, part_ml [B, H, S, 2] fp32 with S = fa_decode_num_splits(Lmax, num_splits)."""
+    import torch
+    B, H, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query per (batch, head)")
+    Lmax = k_cache.shape[2]
+    S = fa_decode_num_splits(Lmax, num_splits)
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k_cache, "k_cache", torch.bfloat16, dev, (B, H, Lmax, d))
+    _need(v_cache, "v_cache", torch.bfloat16, dev, (B, H, Lmax, d))
+    _need(seqlens, "seqlens", torch.int32, dev, (B,))
+    _need(part_o, "part_o", torch.float32, dev, (B, H, S, d))
+    _need(part_ml, "part_ml", torch.float32, dev, (B, H, S, 2))
+    _check(lib().fa_decode_partials(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(part_o),
+                                    _ptr(part_ml), B, H, d, _scale(scale, d), int(num_splits), _stream_ptr(stream)),
+           "fa_decode_partials")
+
+
+def fa_decode_merge(part_o, part_ml, o, lse=None, stream=None) -> None:
+    """Merge R groups of S partials, part_o [R, B, H, S, d] and part_ml [R, B, H, S, 2] fp32, into o [B, H, 1, d]
+    bf16 and lse [B, H] (see include/fa.h: fa_decode_merge)."""
+    import torch
+    R, B, H, S, d = part_o.shape
+    dev = part_o.device
+    _need(part_o, "part_o", torch.float32, dev)
+    _need(part_ml, "part_ml", torch.float32, dev, (R, B, H, S, 2))
+    _need(o, "o", torch.bfloat16, dev, (B, H, 1, d))
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev, (B, H))
+    _check(lib().fa_decode_merge(_ptr(part_o), _ptr(part_ml), R, S, _ptr(o), _ptr(lse), B, H, d,
+                                 _stream_ptr(stream)), "fa_decode_merge")
 
 
 def fa_get_device_error(stream=None) -> int:

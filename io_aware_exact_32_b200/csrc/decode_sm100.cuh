@@ -225,29 +225,34 @@ __global__ void __launch_bounds__(DecTraits<D>::THREADS) fa_decode_split_kernel(
 
 // Reduce the S partials of each (batch, head): one warp per (batch, head).
 template <int D>
+// Partials come in R groups (R = 1 for one device; R ranks after an all-gather of per-rank
+// partials in sequence-parallel decode): partial s of group r for (b, h) sits at row
+// (r * BH + bh) * S + s.
 __global__ void __launch_bounds__(128) fa_decode_merge_kernel(const float* __restrict__ part_o,
                                                               const float* __restrict__ part_ml,
                                                               __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-                                                              int BH, int S) {
+                                                              int BH, int S, int R = 1) {
   constexpr int PER = D / 32;
   const int bh = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (bh >= BH) return;
-  const float* ml = part_ml + (size_t)bh * S * 2;
+  auto row = [&](int i) { return ((size_t)(i / S) * BH + bh) * S + i % S; };  // i = r * S + s
+  const int n = R * S;
   float mt = -INFINITY;
-  for (int s = lane; s < S; s += 32) mt = fmaxf(mt, ml[2 * s]);
+  for (int i = lane; i < n; i += 32) mt = fmaxf(mt, part_ml[2 * row(i)]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
   const float base = (mt == -INFINITY) ? 0.f : mt;
   float l = 0.f, acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  for (int s = 0; s < S; ++s) {
-    const float ms = ml[2 * s];
+  for (int i = 0; i < n; ++i) {
+    const size_t ri = row(i);
+    const float ms = part_ml[2 * ri];
     if (ms == -INFINITY) continue;
     const float w = ex2_approx(ms - base);
-    l += w * ml[2 * s + 1];
-    const float* po = part_o + ((size_t)bh * S + s) * D + lane * PER;
+    l += w * part_ml[2 * ri + 1];
+    const float* po = part_o + ri * D + lane * PER;
 #pragma unroll
     for (int e = 0; e < PER; ++e) acc[e] = fmaf(w, po[e], acc[e]);
   }

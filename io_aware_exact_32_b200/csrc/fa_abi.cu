@@ -253,6 +253,30 @@ fa_status launch_decode(const void* q, const void* kc, const void* vc, const int
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+template <int D>
+fa_status launch_decode_partials(const void* q, const void* kc, const void* vc, const int* seqlens, int Lmax,
+                                 float* part_o, float* part_ml, int BH, int H, float scale, int S,
+                                 cudaStream_t stream) {
+  using T = fa::DecTraits<D>;
+  if (!set_smem(fa::fa_decode_split_kernel<D>, T::SMEM_BYTES)) return FA_ERR_CUDA;
+  fa::DecParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<const __nv_bfloat16*>(kc);
+  p.vc = static_cast<const __nv_bfloat16*>(vc);
+  p.seqlens = seqlens;
+  p.part_o = part_o;
+  p.part_ml = part_ml;
+  p.Lmax = Lmax;
+  p.H = H;
+  p.S = S;
+  p.C = decode_chunk(Lmax, S);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const long long units = (long long)BH * S;
+  if (units > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  fa::fa_decode_split_kernel<D><<<(unsigned)units, T::THREADS, T::SMEM_BYTES, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
@@ -349,6 +373,53 @@ fa_status fa_decode_splitkv(const void* q, const void* k_cache, const void* v_ca
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 64 ? launch_decode<64>(q, k_cache, v_cache, seqlens, Lmax, o, lse, (int)BH, H, scale, S, workspace, s)
                  : launch_decode<128>(q, k_cache, v_cache, seqlens, Lmax, o, lse, (int)BH, H, scale, S, workspace, s);
+}
+
+int fa_decode_num_splits(int Lmax, int num_splits) {
+  if (Lmax < 1 || Lmax > kMaxSeq || num_splits < 0 || num_splits > kMaxSplits) return 0;
+  return decode_splits(Lmax, num_splits);
+}
+
+fa_status fa_decode_partials(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, int Lmax,
+                             float* part_o, float* part_ml, int B, int H, int d, float scale, int num_splits,
+                             void* stream) {
+  if (B < 0 || H < 0 || num_splits < 0) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (Lmax < 1 || Lmax > kMaxSeq) return Lmax < 1 ? FA_ERR_INVALID_ARG : FA_ERR_UNSUPPORTED;
+  if (num_splits > kMaxSplits) return FA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  if (BH == 0) return FA_OK;
+  if (!q || !k_cache || !v_cache || !seqlens || !part_o || !part_ml) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(part_o) || !aligned16(part_ml) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return FA_ERR_MISALIGNED;
+  const int S = decode_splits(Lmax, num_splits);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode_partials<64>(q, k_cache, v_cache, seqlens, Lmax, part_o, part_ml, (int)BH, H, scale, S, s)
+                 : launch_decode_partials<128>(q, k_cache, v_cache, seqlens, Lmax, part_o, part_ml, (int)BH, H, scale, S,
+                                               s);
+}
+
+fa_status fa_decode_merge(const float* part_o, const float* part_ml, int R, int S, void* o, float* lse, int B, int H,
+                          int d, void* stream) {
+  if (B < 0 || H < 0 || R < 1 || S < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH > 0x7fffffffLL || (long long)R * S > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  if (BH == 0) return FA_OK;
+  if (!part_o || !part_ml || !o) return FA_ERR_INVALID_ARG;
+  if (!aligned16(part_o) || !aligned16(part_ml) || !aligned16(o) || (lse && !aligned16(lse))) return FA_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned grid = (unsigned)((BH + 3) / 4);
+  if (d == 64)
+    fa::fa_decode_merge_kernel<64><<<grid, 128, 0, s>>>(part_o, part_ml, static_cast<__nv_bfloat16*>(o), lse,
+                                                        (int)BH, S, R);
+  else
+    fa::fa_decode_merge_kernel<128><<<grid, 128, 0, s>>>(part_o, part_ml, static_cast<__nv_bfloat16*>(o), lse,
+                                                         (int)BH, S, R);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status fa_get_device_error(void* stream) {
