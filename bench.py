@@ -30,6 +30,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -103,10 +104,12 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, path: str | None = None):
         self.gpu = str(gpu_index)
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        # The raw samples are kept where --clock-log asks (else a temporary file); the summary
+        # goes into the JSON line either way.
+        self.path = path or os.path.join(tempfile.gettempdir(), f"clocks_bench_{os.getpid()}.csv")
 
     def start(self):
         try:
@@ -292,7 +295,7 @@ def run_ours(args):
 
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    clocks = ClockSampler(dev.index if world == 1 else local).start() if rank == 0 else None
+    clocks = ClockSampler(dev.index if world == 1 else local, args.clock_log).start() if rank == 0 else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -603,6 +606,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--clock-log", default=None, help="CSV file for the raw nvidia-smi clock samples")
     ap.add_argument("--no-extra", action="store_true", help="skip the d=128 and decode side measurements")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches instead of a replayed CUDA graph")
     ap.add_argument("--case", choices=CASES, default=None,

@@ -26,7 +26,7 @@ section):
 * "Transformer、注意力机制与优化", section Flash-Decoding: a single query
   attends to every cached key/value of its sequence.
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
 
 * ``scale`` is an explicit argument; the pages use 1/sqrt(d).
 * Causal alignment when Nq != Nk is bottom-right: key j is visible to query i
