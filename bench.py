@@ -519,6 +519,30 @@ def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
                                     "fwd_frac_of_2250": fwd_t / 2250.0, "bwd_tflops": fb / t_b / 1e12,
                                     "fwd_bwd_tflops": fb_t, "fwd_bwd_frac": fb_t / peaks["bf16_tflops"],
                                     "fwd_bwd_frac_of_2250": fb_t / 2250.0, "fwd_ms": 1e3 * t_f, "bwd_ms": 1e3 * t_b}
+        # FP8 forward on the same inputs: Q and K rotated (random-sign Hadamard) and quantised, V quantised.
+        signs = W.make_hadamard_signs(cfg.d, 11).to(dev)
+        q8, dsq = fa.quantize_fp8(q, signs, True, stream)
+        k8, dsk = fa.quantize_fp8(k, signs, True, stream)
+        v8, dsv = fa.quantize_fp8(v, None, False, stream)
+        o8 = torch.empty_like(o)
+        lse8 = torch.empty_like(lse)
+        t_f8 = timed(lambda: fa.fa_fwd_fp8(q8, k8, v8, dsq, dsk, dsv, o8, lse8, True, cfg.scale, stream))
+
+        def quantize_all():
+            fa.fa_quantize_fp8(q, signs, q8, dsq, True, stream)
+            fa.fa_quantize_fp8(k, signs, k8, dsk, True, stream)
+            fa.fa_quantize_fp8(v, None, v8, dsv, False, stream)
+
+        t_q8 = timed(quantize_all)
+        f8_t = ff / t_f8 / 1e12
+        qbytes = 3 * q.numel() * 3  # algorithmic: read bf16 (2 B) and write E4M3 (1 B) for Q, K, V
+        res[f"fp8_causal_n{n}_d128"] = {
+            "fwd_tflops": f8_t, "fwd_ms": 1e3 * t_f8, "vs_bf16_fwd": t_f / t_f8,
+            "fwd_frac_of_fp8_peak": f8_t / (2.0 * peaks["bf16_tflops"]), "fwd_frac_of_4500": f8_t / 4500.0,
+            "fp8_peak_note": "2 x measured bf16 (the nominal fp8 / bf16 ratio)",
+            "quantize_qkv_ms": 1e3 * t_q8, "quantize_gbs_algorithmic": qbytes / t_q8 / 1e9,
+            "fwd_incl_quantize_tflops": ff / (t_f8 + t_q8) / 1e12}
+        del q8, k8, v8, dsq, dsk, dsv, o8, lse8
         if n == 4096:
             t_bd = timed(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, True, cfg.scale, stream,
                                            deterministic=True))
@@ -540,7 +564,7 @@ def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
     return res
 
 
-CASES = ("fwd_c2", "bwd_c2", "fwd_n4096_d128", "bwd_n4096_d128", "decode")
+CASES = ("fwd_c2", "bwd_c2", "fwd_n4096_d128", "bwd_n4096_d128", "fwd_fp8_n4096_d128", "decode")
 
 
 def run_case(args):
@@ -570,7 +594,14 @@ def run_case(args):
         x = W.make_config_inputs(cfg)
         q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
         o, lse = fa.attention_forward(q, k, v, causal=causal, scale=cfg.scale)
-        if name.startswith("fwd"):
+        if name.startswith("fwd_fp8"):
+            signs = W.make_hadamard_signs(cfg.d, 11).to(dev)
+            q8, dsq = fa.quantize_fp8(q, signs, True, stream)
+            k8, dsk = fa.quantize_fp8(k, signs, True, stream)
+            v8, dsv = fa.quantize_fp8(v, None, False, stream)
+            fn = lambda: fa.fa_fwd_fp8(q8, k8, v8, dsq, dsk, dsv, o, lse, causal, cfg.scale, stream)
+            units = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal) / 1e12
+        elif name.startswith("fwd"):
             fn = lambda: fa.fa_fwd(q, k, v, o, lse, causal, cfg.scale, stream)
             units = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal) / 1e12
         else:

@@ -82,6 +82,45 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
                  void* stream);
 
 /*
+ * FP8 (E4M3) operands with incoherent processing ("FlashAttention 系列技术详解",
+ * section 具体技术, FlashAttention-3): the score and output GEMMs run on FP8
+ * tensor cores, and Q and K are first multiplied by a random orthogonal matrix,
+ * a Hadamard transform, to spread outlier channels before quantisation.
+ *
+ * E4M3 here is the "FN" byte format: 1 sign, 4 exponent bits (bias 7),
+ * 3 mantissa bits, largest finite value 448, no infinities; conversions round
+ * to nearest even and saturate.
+ *
+ * fa_quantize_fp8: x8 = rn_e4m3(y * 448 / amax) per (batch, head), where
+ *   y = H_d (s o x_row) for every row when hadamard != 0 (H_d the Sylvester
+ *   Hadamard matrix, s the signs; all in fp32), y = x_row otherwise, and amax
+ *   is the largest |y| of the head.  descale[b, h] = (amax / 448) / sqrt(d)
+ *   with the rotation, amax / 448 without, so that x M ~= x8 * descale with
+ *   M = diag(s) H_d / sqrt(d) orthogonal.  Rotate Q and K with the same signs
+ *   (Q M (K M)^T = Q K^T); quantise V with hadamard = 0.
+ *   x       [B, H, N, d] bf16, read
+ *   signs   [d] fp32 of +-1, read; NULL = all +1 (plain Hadamard)
+ *   x8      [B, H, N, d] E4M3 bytes, written
+ *   descale [B, H] fp32, written (also used as scratch during the call)
+ *   d in {64, 128}; N == 0 writes descale = 0.  x and x8 16-byte aligned,
+ *   signs and descale 4-byte aligned.
+ *
+ * fa_fwd_fp8: the forward of fa_fwd on E4M3 operands, O = softmax(scale * Qd Kd^T
+ *   [+ causal mask]) Vd with Qd = q8 * descale_q[b, h] (likewise K, V).  The
+ *   softmax weights are rounded to E4M3 for the P V product and O is normalised
+ *   by the sum of the rounded weights; LSE uses the exact fp32 sum.
+ *   q8 [B, H, Nq, d], k8 / v8 [B, H, Nk, d] E4M3 bytes; descale_* [B, H] fp32;
+ *   o [B, H, Nq, d] bf16 and lse [B, H, Nq] fp32 written as in fa_fwd.
+ *   d = 128 only (FA_ERR_UNSUPPORTED otherwise); other limits as fa_fwd.
+ */
+FA_API fa_status fa_quantize_fp8(const void* x, const float* signs, void* x8, float* descale,
+                 int B, int H, int N, int d, int hadamard, void* stream);
+FA_API fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                 const float* descale_q, const float* descale_k, const float* descale_v,
+                 void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale,
+                 int causal, void* stream);
+
+/*
  * Bytes of fp32 workspace fa_bwd needs: D [B, H, Nq] plus the dQ accumulator
  * [B, H, Nq, d], each region 256-byte aligned.  Returns 0 on invalid sizes.
  */

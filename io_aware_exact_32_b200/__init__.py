@@ -8,10 +8,10 @@ and raises on a non-zero status.  PyTorch provides device memory and streams.
 C-ABI mirrors (same names, torch tensors in place of pointers):
     fa_fwd, fa_bwd, fa_bwd_deterministic, fa_bwd_workspace_size, fa_decode_splitkv, fa_decode_num_splits,
     fa_decode_partials, fa_decode_merge,
-    fa_decode_workspace_size, fa_decode_splitkv_noalloc, fa_get_device_error,
-    fa_status_string, fa_version
+    fa_decode_workspace_size, fa_decode_splitkv_noalloc, fa_quantize_fp8, fa_fwd_fp8,
+    fa_get_device_error, fa_status_string, fa_version
 Convenience wrappers that allocate outputs:
-    attention_forward, attention_backward, decode_splitkv
+    attention_forward, attention_backward, decode_splitkv, quantize_fp8, attention_forward_fp8
 """
 from __future__ import annotations
 
@@ -23,8 +23,9 @@ __all__ = [
     "FAError", "lib", "lib_path",
     "fa_fwd", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size", "fa_decode_splitkv",
     "fa_decode_workspace_size", "fa_decode_num_splits", "fa_decode_partials", "fa_decode_merge",
-    "fa_decode_splitkv_noalloc", "fa_get_device_error", "fa_status_string", "fa_version",
-    "attention_forward", "attention_backward", "decode_splitkv",
+    "fa_decode_splitkv_noalloc", "fa_quantize_fp8", "fa_fwd_fp8", "fa_get_device_error", "fa_status_string",
+    "fa_version", "attention_forward", "attention_backward", "decode_splitkv", "quantize_fp8",
+    "attention_forward_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -73,6 +74,10 @@ def lib() -> ctypes.CDLL:
     L.fa_decode_partials.restype = i
     L.fa_decode_merge.argtypes = [vp, vp, i, i, vp, vp, i, i, i, vp]
     L.fa_decode_merge.restype = i
+    L.fa_quantize_fp8.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp]
+    L.fa_quantize_fp8.restype = i
+    L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    L.fa_fwd_fp8.restype = i
     L.fa_get_device_error.argtypes = [vp]
     L.fa_get_device_error.restype = i
     L.fa_status_string.argtypes = [i]
@@ -262,6 +267,47 @@ def fa_decode_merge(part_o, part_ml, o, lse=None, stream=None) -> None:
                                  _stream_ptr(stream)), "fa_decode_merge")
 
 
+def _need_e4m3(t, name, device, shape=None):
+    """E4M3 codes: a torch.uint8 or torch.float8_e4m3fn tensor."""
+    import torch
+    dtype = t.dtype if isinstance(t, torch.Tensor) and t.dtype in (torch.uint8, torch.float8_e4m3fn) else torch.uint8
+    _need(t, name, dtype, device, shape)
+
+
+def fa_quantize_fp8(x, signs, x8, descale, hadamard: bool = True, stream=None) -> None:
+    """Per-head E4M3 quantisation with optional incoherent processing (see include/fa.h: fa_quantize_fp8).
+    x [B,H,N,d] bf16, signs [d] fp32 (+-1) or None, x8 [B,H,N,d] uint8 / float8_e4m3fn, descale [B,H] fp32."""
+    import torch
+    B, H, N, d = x.shape
+    dev = x.device
+    _need(x, "x", torch.bfloat16, dev)
+    if signs is not None:
+        _need(signs, "signs", torch.float32, dev, (d,))
+    _need_e4m3(x8, "x8", dev, (B, H, N, d))
+    _need(descale, "descale", torch.float32, dev, (B, H))
+    _check(lib().fa_quantize_fp8(_ptr(x), _ptr(signs), _ptr(x8), _ptr(descale), B, H, N, d, int(bool(hadamard)),
+                                 _stream_ptr(stream)), "fa_quantize_fp8")
+
+
+def fa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, causal: bool, scale=None, stream=None) -> None:
+    """Forward on E4M3 operands (see include/fa.h: fa_fwd_fp8).  q8 [B,H,Nq,d], k8/v8 [B,H,Nk,d] uint8 or
+    float8_e4m3fn codes; descale_* [B,H] fp32; o [B,H,Nq,d] bf16, lse [B,H,Nq] fp32."""
+    import torch
+    B, H, Nq, d = q8.shape
+    Nk = k8.shape[2]
+    dev = q8.device
+    _need_e4m3(q8, "q8", dev)
+    _need_e4m3(k8, "k8", dev, (B, H, Nk, d))
+    _need_e4m3(v8, "v8", dev, (B, H, Nk, d))
+    for t, n in ((descale_q, "descale_q"), (descale_k, "descale_k"), (descale_v, "descale_v")):
+        _need(t, n, torch.float32, dev, (B, H))
+    _need(o, "o", torch.bfloat16, dev, (B, H, Nq, d))
+    _need(lse, "lse", torch.float32, dev, (B, H, Nq))
+    _check(lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v),
+                            _ptr(o), _ptr(lse), B, H, Nq, Nk, d, _scale(scale, d), int(bool(causal)),
+                            _stream_ptr(stream)), "fa_fwd_fp8")
+
+
 def fa_get_device_error(stream=None) -> int:
     return int(lib().fa_get_device_error(_stream_ptr(stream)))
 
@@ -306,4 +352,28 @@ def decode_splitkv(q, k_cache, v_cache, seqlens, scale=None, num_splits: int = 0
     if workspace is None:
         workspace = _workspace(fa_decode_workspace_size(B, H, k_cache.shape[2], d, num_splits), q.device)
     fa_decode_splitkv(q, k_cache, v_cache, seqlens, o, lse, workspace, scale, num_splits, stream)
+    return o, lse
+
+
+def quantize_fp8(x, signs=None, hadamard: bool = True, stream=None):
+    """Allocate the codes and scales and run fa_quantize_fp8; returns (x8 uint8, descale fp32 [B, H])."""
+    import torch
+    B, H, N, d = x.shape
+    x8 = torch.empty((B, H, N, d), dtype=torch.uint8, device=x.device)
+    descale = torch.empty((B, H), dtype=torch.float32, device=x.device)
+    fa_quantize_fp8(x, signs, x8, descale, hadamard, stream)
+    return x8, descale
+
+
+def attention_forward_fp8(q, k, v, causal: bool = False, scale=None, signs=None, hadamard: bool = True, stream=None):
+    """FP8 forward from bf16 Q, K, V: Q and K are rotated (random-sign Hadamard, the same signs for both)
+    and quantised, V is quantised, then fa_fwd_fp8 runs.  Returns (o bf16, lse fp32)."""
+    import torch
+    B, H, Nq, d = q.shape
+    q8, dq = quantize_fp8(q, signs, hadamard, stream)
+    k8, dk = quantize_fp8(k, signs, hadamard, stream)
+    v8, dv = quantize_fp8(v, None, False, stream)
+    o = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    fa_fwd_fp8(q8, k8, v8, dq, dk, dv, o, lse, causal, scale, stream)
     return o, lse

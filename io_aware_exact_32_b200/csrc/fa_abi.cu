@@ -13,6 +13,7 @@
 #include "bwd_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "fwd_sm100.cuh"
+#include "quant_sm100.cuh"
 
 namespace {
 
@@ -36,16 +37,19 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [BH, N, D] bf16 viewed as a 3-D tensor {D, N, BH}; box = 64 columns x 128 rows x 1, 128-byte swizzle.
-// Rows past N read as zero.
-bool make_map_3d(CUtensorMap* map, const void* base, int D, int N, long long BH) {
+// [BH, N, D] bf16 (or 1-byte E4M3 when f8) viewed as a 3-D tensor {D, N, BH}; box = one 128-byte
+// row segment (64 bf16 or 128 E4M3 columns) x 128 rows x 1, 128-byte swizzle.  Rows past N read
+// as zero.
+bool make_map_3d(CUtensorMap* map, const void* base, int D, int N, long long BH, bool f8 = false) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
+  const cuuint64_t eb = f8 ? 1 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)D * eb, (cuuint64_t)N * D * eb};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / eb), 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(map, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -119,15 +123,20 @@ int decode_chunk(int Lmax, int S) {
   return (c + 31) & ~31;
 }
 
-template <int D>
+template <int D, bool F8 = false>
 fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int Nq, int Nk,
-                     float scale, int causal, cudaStream_t stream) {
-  using T = fa::FwdTraits<D>;
+                     float scale, int causal, cudaStream_t stream, const float* descale_q = nullptr,
+                     const float* descale_k = nullptr, const float* descale_v = nullptr) {
+  using T = fa::FwdTraits<D, F8>;
   CUtensorMap mq, mk, mv;
-  if (!make_map_3d(&mq, q, D, Nq, BH) || !make_map_3d(&mk, k, D, Nk, BH) || !make_map_3d(&mv, v, D, Nk, BH))
+  if (!make_map_3d(&mq, q, D, Nq, BH, F8) || !make_map_3d(&mk, k, D, Nk, BH, F8) ||
+      !make_map_3d(&mv, v, D, Nk, BH, F8))
     return FA_ERR_CUDA;
-  if (!set_smem(fa::fa_fwd_kernel<D>, T::SMEM_BYTES)) return FA_ERR_CUDA;
+  if (!set_smem(fa::fa_fwd_kernel<D, F8>, T::SMEM_BYTES)) return FA_ERR_CUDA;
   fa::FwdParams p;
+  p.descale_q = descale_q;
+  p.descale_k = descale_k;
+  p.descale_v = descale_v;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.Nq = Nq;
@@ -140,7 +149,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   p.causal = causal ? 1 : 0;
   const long long blocks = (long long)p.nunits * BH;
   if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  fa::fa_fwd_kernel<D><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  fa::fa_fwd_kernel<D, F8><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -300,6 +309,69 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   }
   return d == 64 ? launch_fwd<64>(q, k, v, o, lse, (int)BH, Nq, Nk, scale, causal, s)
                  : launch_fwd<128>(q, k, v, o, lse, (int)BH, Nq, Nk, scale, causal, s);
+}
+
+fa_status fa_quantize_fp8(const void* x, const float* signs, void* x8, float* descale, int B, int H, int N, int d,
+                          int hadamard, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (N > kMaxSeq || (long long)B * H > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH == 0) return FA_OK;
+  if (!descale || (N > 0 && (!x || !x8))) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(descale) & 3u) || (signs && (reinterpret_cast<uintptr_t>(signs) & 3u)) ||
+      (N > 0 && (!aligned16(x) || !aligned16(x8))))
+    return FA_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The descale buffer first holds the per-head amax (float bits, atomically maximised).
+  if (cudaMemsetAsync(descale, 0, (size_t)BH * sizeof(float), s) != cudaSuccess) return FA_ERR_CUDA;
+  if (N > 0) {
+    const int chunks = (N + fa::kQuantRowsPerBlock - 1) / fa::kQuantRowsPerBlock;
+    const long long blocks = BH * chunks;
+    if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    uint8_t* out = static_cast<uint8_t*>(x8);
+    const int had = hadamard ? 1 : 0;
+    if (d == 64) {
+      fa::fa_quant_amax_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(xb, signs, reinterpret_cast<unsigned*>(descale), N,
+                                                                     chunks, had);
+      fa::fa_quant_store_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(xb, signs, descale, out, N, chunks, had);
+    } else {
+      fa::fa_quant_amax_kernel<128><<<(unsigned)blocks, 256, 0, s>>>(xb, signs, reinterpret_cast<unsigned*>(descale),
+                                                                      N, chunks, had);
+      fa::fa_quant_store_kernel<128><<<(unsigned)blocks, 256, 0, s>>>(xb, signs, descale, out, N, chunks, had);
+    }
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+  const float r = hadamard ? (float)(1.0 / std::sqrt((double)d)) : 1.f;
+  fa::fa_quant_descale_kernel<<<(unsigned)((BH + 255) / 256), 256, 0, s>>>(descale, BH, r);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* descale_q, const float* descale_k,
+                     const float* descale_v, void* o, float* lse, int B, int H, int Nq, int Nk, int d, float scale,
+                     int causal, void* stream) {
+  fa_status st = check_common(B, H, Nq, Nk, d, scale);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  const long long BH = (long long)B * H;
+  if (BH == 0 || Nq == 0) return FA_OK;
+  if (!q8 || !o || !lse || !descale_q || (Nk > 0 && (!k8 || !v8 || !descale_k || !descale_v)))
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(o) || !aligned16(lse) || (Nk > 0 && (!aligned16(k8) || !aligned16(v8))) ||
+      (reinterpret_cast<uintptr_t>(descale_q) & 3u) || (reinterpret_cast<uintptr_t>(descale_k) & 3u) ||
+      (reinterpret_cast<uintptr_t>(descale_v) & 3u))
+    return FA_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (Nk == 0) {
+    const long long rows = BH * Nq;
+    const long long n = rows * d;
+    fa::fa_fwd_empty_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(static_cast<__nv_bfloat16*>(o), lse, rows,
+                                                                         d);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  }
+  return launch_fwd<128, true>(q8, k8, v8, o, lse, (int)BH, Nq, Nk, scale, causal, s, descale_q, descale_k,
+                               descale_v);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int Nq, int d) {

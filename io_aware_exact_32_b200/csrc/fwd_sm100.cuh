@@ -42,15 +42,19 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #endif
 constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
 
-template <int D>
+template <int D, bool F8 = false>
 struct FwdTraits {
   static_assert(D == 64 || D == 128, "head dim");
+  static_assert(!F8 || D == 128, "FP8 operands: d = 128");
+  static constexpr int EB = F8 ? 1 : 2;                // bytes per Q/K/V element (E4M3 or bf16)
   static constexpr int BM = 128;                       // query rows per tile
   static constexpr int BN = 128;                       // keys per tile
-  static constexpr int NBOX = D / 64;                  // 64-column TMA boxes per tile
-  static constexpr int BOX_BYTES = 128 * 64 * 2;       // 16 KB
-  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128 x D bf16 tile
-  static constexpr int NS = (D == 64) ? 6 : 3;         // K/V ring stages
+  static constexpr int BOX_COLS = 128 / EB;            // elements per 128-byte swizzle row
+  static constexpr int NBOX = D * EB / 128;            // 128-byte-wide TMA boxes per tile
+  static constexpr int BOX_BYTES = 128 * 128;          // 128 rows x 128 bytes = 16 KB
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128 x D tile
+  static constexpr int KSTEP = 32 / EB;                // MMA K per instruction (32 bytes of operand)
+  static constexpr int NS = F8 ? 8 : ((D == 64) ? 6 : 3);  // K/V ring stages
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 2 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
@@ -71,8 +75,8 @@ struct FwdTraits {
   static __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }
   static __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + (uint32_t)D * t; }
   static constexpr int THREADS = 320;  // warps 0-7 softmax, 8 MMA issuer, 9 TMA
-  static constexpr uint32_t IDESC_QK = make_idesc_bf16(128, 128, false, false);
-  static constexpr uint32_t IDESC_PV = make_idesc_bf16(128, D, false, true);
+  static constexpr uint32_t IDESC_QK = F8 ? make_idesc_e4m3(128, 128, false, false) : make_idesc_bf16(128, 128, false, false);
+  static constexpr uint32_t IDESC_PV = F8 ? make_idesc_e4m3(128, D, false, true) : make_idesc_bf16(128, D, false, true);
 };
 
 struct FwdParams {
@@ -84,6 +88,10 @@ struct FwdParams {
                      // the two softmax groups split that tile's key tiles: even / odd)
   float scale_log2;  // scale * log2(e)
   int causal;
+  // FP8 operands only: per-(batch, head) dequantisation factors (x = x8 * descale).
+  const float* descale_q;
+  const float* descale_k;
+  const float* descale_v;
 };
 
 // Number of 128-key tiles the CTA owning query rows [q0, q0 + span) must visit.
@@ -96,27 +104,34 @@ __device__ __forceinline__ int fwd_num_kv_tiles(int q0, int span, int Nq, int Nk
   return min(nkt, kmax / 128 + 1);
 }
 
-template <int D>
+template <int D, bool F8>
 __device__ __forceinline__ void fwd_issue_qk(uint32_t tmem_d, uint32_t q_smem, uint32_t k_smem) {
-  using T = FwdTraits<D>;
+  using T = FwdTraits<D, F8>;
   const uint64_t qd = make_sdesc_sw128(q_smem, 16, 1024), kd = make_sdesc_sw128(k_smem, 16, 1024);
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    // K advances 16 elements (32 bytes) inside a 128-byte swizzle row; every 4 steps, the next box.
+  for (int kk = 0; kk < D / T::KSTEP; ++kk) {
+    // K advances 32 bytes inside a 128-byte swizzle row; every 4 steps, the next box.
     const uint64_t off = (uint64_t)(((kk / 4) * T::BOX_BYTES + (kk % 4) * 32) >> 4);
-    mma_ss_w(tmem_d, qd + off, kd + off, T::IDESC_QK, kk > 0 ? 1u : 0u);
+    if constexpr (F8)
+      mma_ss_w_f8(tmem_d, qd + off, kd + off, T::IDESC_QK, kk > 0 ? 1u : 0u);
+    else
+      mma_ss_w(tmem_d, qd + off, kd + off, T::IDESC_QK, kk > 0 ? 1u : 0u);
   }
 }
 
-template <int D>
+template <int D, bool F8>
 __device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
-  using T = FwdTraits<D>;
+  using T = FwdTraits<D, F8>;
   const uint64_t vd = make_sdesc_sw128(v_smem, T::BOX_BYTES, 1024);
 #pragma unroll
-  for (int kk = 0; kk < 128 / 16; ++kk) {
-    // 16 keys per step: P columns advance by 8 (two bf16 per 32-bit column), V rows by 16 x 128 B.
-    mma_ts_w(tmem_d, tmem_p + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), T::IDESC_PV,
-           (accumulate || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < 128 / T::KSTEP; ++kk) {
+    // KSTEP keys per step: P advances 8 32-bit columns (two bf16 or four E4M3 per column), V rows
+    // by KSTEP x 128 bytes.
+    const uint64_t voff = (uint64_t)((kk * T::KSTEP * 128) >> 4);
+    if constexpr (F8)
+      mma_ts_w_f8(tmem_d, tmem_p + kk * 8, vd + voff, T::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+    else
+      mma_ts_w(tmem_d, tmem_p + kk * 8, vd + voff, T::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -142,11 +157,11 @@ __device__ __forceinline__ float max64(const float* s) {
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-template <int D>
-__global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
+template <int D, bool F8 = false>
+__global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using T = FwdTraits<D>;
+  using T = FwdTraits<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -206,7 +221,9 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
     int kmax = p.Nk - 1;  // last visible key of this row (inclusive)
     if (p.causal) kmax = min(kmax, row + p.Nk - p.Nq);
     float m_run = -INFINITY, l_run = 0.f, lr_run = 0.f;
-    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+    float scale_log2 = p.scale_log2;
+    if constexpr (F8) scale_log2 *= __ldg(p.descale_q + bh) * __ldg(p.descale_k + bh);
+    const float2 sc2 = make_float2(scale_log2, scale_log2);
     bool ok = true;
     for (int step = 0; step < n_own; ++step) {
       const int j = two ? step : 2 * step + t;  // key tile
@@ -235,7 +252,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
           if (c + 64 > lim) s2[c] = -INFINITY;
       }
       const float mx = fmaxf(mx_a, max64(s2));
-      const float m_tile = mx * p.scale_log2;
+      const float m_tile = mx * scale_log2;
       float alpha = 1.f;
       bool resc = false;
       if (m_tile > m_run + kRescaleThreshold) {
@@ -251,24 +268,47 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       float2 sum_e[2], sum_r[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) sum_e[i] = sum_r[i] = make_float2(0.f, 0.f);
+      if constexpr (F8) {
+        // E4M3 weights, four per 32-bit column (P <= 2^8 stays inside the format's 448).
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const float* src = (ch < 2) ? s + 32 * ch : s2 + 32 * (ch - 2);
-        uint32_t pk[16];
+        for (int ch = 0; ch < 4; ++ch) {
+          const float* src = (ch < 2) ? s + 32 * ch : s2 + 32 * (ch - 2);
+          uint32_t pk[8];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float2 x = ffma2(make_float2(src[2 * c], src[2 * c + 1]), sc2, nb2);
-          float2 e;
-          if (kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-            e = exp2_poly2(x);
-          } else {
-            e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          for (int c = 0; c < 8; ++c) {
+            const float2 x0 = ffma2(make_float2(src[4 * c], src[4 * c + 1]), sc2, nb2);
+            const float2 x1 = ffma2(make_float2(src[4 * c + 2], src[4 * c + 3]), sc2, nb2);
+            const float2 e0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+            const float2 e1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+            const uint32_t lo = f32x2_to_e4m3x2(e0.x, e0.y), hi = f32x2_to_e4m3x2(e1.x, e1.y);
+            pk[c] = lo | (hi << 16);
+            sum_e[0] = fadd2(sum_e[0], e0);
+            sum_e[1] = fadd2(sum_e[1], e1);
+            sum_r[0] = fadd2(sum_r[0], e4m3x2_to_f32x2(lo));
+            sum_r[1] = fadd2(sum_r[1], e4m3x2_to_f32x2(hi));
           }
-          pk[c] = pack_bf16x2(e.x, e.y);
-          sum_e[c & 1] = fadd2(sum_e[c & 1], e);
-          sum_r[c & 1] = fadd2(sum_r[c & 1], make_float2(bf16lo_to_f32(pk[c]), bf16hi_to_f32(pk[c])));
+          tmem_st32x32b_x8(lane_addr + colS + 8 * ch, pk);
         }
-        tmem_st32x32b_x16(lane_addr + colS + 16 * ch, pk);
+      } else {
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const float* src = (ch < 2) ? s + 32 * ch : s2 + 32 * (ch - 2);
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float2 x = ffma2(make_float2(src[2 * c], src[2 * c + 1]), sc2, nb2);
+            float2 e;
+            if (kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
+              e = exp2_poly2(x);
+            } else {
+              e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            }
+            pk[c] = pack_bf16x2(e.x, e.y);
+            sum_e[c & 1] = fadd2(sum_e[c & 1], e);
+            sum_r[c & 1] = fadd2(sum_r[c & 1], make_float2(bf16lo_to_f32(pk[c]), bf16hi_to_f32(pk[c])));
+          }
+          tmem_st32x32b_x16(lane_addr + colS + 16 * ch, pk);
+        }
       }
       const float2 tot_e = fadd2(sum_e[0], sum_e[1]);
       const float2 tot_r = fadd2(sum_r[0], sum_r[1]);
@@ -325,7 +365,9 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
     }
     if (ok && (two || t == 0)) {
       tc_fence_after();
-      const float inv = lr_run > 0.f ? 1.f / lr_run : 0.f;
+      float num = 1.f;
+      if constexpr (F8) num = __ldg(p.descale_v + bh);
+      const float inv = lr_run > 0.f ? num / lr_run : 0.f;
       const bool in_range = row < p.Nq;
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D;
 #pragma unroll
@@ -379,14 +421,14 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
           const bool has1 = 2 * i + 1 < n_kv;
           if (!(ok = warp_wait(bar(T::BAR_KV_FULL + ik0 % T::NS), (ik0 / T::NS) & 1, abort_flag))) break;
           tc_fence_after();
-          fwd_issue_qk<D>(tS[0], q_smem[0], sbase + T::OFF_KV + (ik0 % T::NS) * T::TILE_BYTES);
+          fwd_issue_qk<D, F8>(tS[0], q_smem[0], sbase + T::OFF_KV + (ik0 % T::NS) * T::TILE_BYTES);
           mma_commit_w(bar(T::BAR_S_FULL + 0));
           release(ik0);
           if (v1_prev >= 0) {
             if (!(ok = warp_wait(bar(T::BAR_KV_FULL + v1_prev % T::NS), (v1_prev / T::NS) & 1, abort_flag))) break;
             if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (i - 1) & 1, abort_flag))) break;
             tc_fence_after();
-            fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v1_prev % T::NS) * T::TILE_BYTES, i - 1 > 0);
+            fwd_issue_pv<D, F8>(tO[1], tS[1], sbase + T::OFF_KV + (v1_prev % T::NS) * T::TILE_BYTES, i - 1 > 0);
             mma_commit_w(bar(T::BAR_O_DONE + 1));
             release(v1_prev);
             v1_prev = -1;
@@ -394,7 +436,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
           if (has1) {
             if (!(ok = warp_wait(bar(T::BAR_KV_FULL + ik1 % T::NS), (ik1 / T::NS) & 1, abort_flag))) break;
             tc_fence_after();
-            fwd_issue_qk<D>(tS[1], q_smem[0], sbase + T::OFF_KV + (ik1 % T::NS) * T::TILE_BYTES);
+            fwd_issue_qk<D, F8>(tS[1], q_smem[0], sbase + T::OFF_KV + (ik1 % T::NS) * T::TILE_BYTES);
             mma_commit_w(bar(T::BAR_S_FULL + 1));
             release(ik1);
             v1_prev = iv1;
@@ -402,7 +444,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
           if (!(ok = warp_wait(bar(T::BAR_KV_FULL + iv0 % T::NS), (iv0 / T::NS) & 1, abort_flag))) break;
           if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), i & 1, abort_flag))) break;
           tc_fence_after();
-          fwd_issue_pv<D>(tO[0], tS[0], sbase + T::OFF_KV + (iv0 % T::NS) * T::TILE_BYTES, i > 0);
+          fwd_issue_pv<D, F8>(tO[0], tS[0], sbase + T::OFF_KV + (iv0 % T::NS) * T::TILE_BYTES, i > 0);
           mma_commit_w(bar(T::BAR_O_DONE + 0));
           release(iv0);
         }
@@ -411,7 +453,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
           if ((ok = warp_wait(bar(T::BAR_KV_FULL + v1_prev % T::NS), (v1_prev / T::NS) & 1, abort_flag)) &&
               (ok = warp_wait(bar(T::BAR_P_READY + 1), i & 1, abort_flag))) {
             tc_fence_after();
-            fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v1_prev % T::NS) * T::TILE_BYTES, i > 0);
+            fwd_issue_pv<D, F8>(tO[1], tS[1], sbase + T::OFF_KV + (v1_prev % T::NS) * T::TILE_BYTES, i > 0);
             mma_commit_w(bar(T::BAR_O_DONE + 1));
           }
         }
@@ -423,28 +465,28 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
         const uint32_t v_smem = sbase + T::OFF_KV + sv * T::TILE_BYTES;
         if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sk), (ik / T::NS) & 1, abort_flag))) break;
         tc_fence_after();
-        fwd_issue_qk<D>(tS[0], q_smem[0], k_smem);
+        fwd_issue_qk<D, F8>(tS[0], q_smem[0], k_smem);
         mma_commit_w(bar(T::BAR_S_FULL + 0));
         if (j > 0) {
           if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (j - 1) & 1, abort_flag))) break;
           tc_fence_after();
-          fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, j - 1 > 0);
+          fwd_issue_pv<D, F8>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, j - 1 > 0);
           mma_commit_w(bar(T::BAR_O_DONE + 1));
           release(v_prev);
         }
-        fwd_issue_qk<D>(tS[1], q_smem[1], k_smem);
+        fwd_issue_qk<D, F8>(tS[1], q_smem[1], k_smem);
         mma_commit_w(bar(T::BAR_S_FULL + 1));
         release(ik);
         if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sv), (iv / T::NS) & 1, abort_flag))) break;
         if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), j & 1, abort_flag))) break;
         tc_fence_after();
-        fwd_issue_pv<D>(tO[0], tS[0], v_smem, j > 0);
+        fwd_issue_pv<D, F8>(tO[0], tS[0], v_smem, j > 0);
         mma_commit_w(bar(T::BAR_O_DONE + 0));
         v_prev = iv;
       }
       if (two && ok && (ok = warp_wait(bar(T::BAR_P_READY + 1), (n_kv - 1) & 1, abort_flag))) {
         tc_fence_after();
-        fwd_issue_pv<D>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, n_kv - 1 > 0);
+        fwd_issue_pv<D, F8>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, n_kv - 1 > 0);
         mma_commit_w(bar(T::BAR_O_DONE + 1));
       }
       if (!ok) {
@@ -462,7 +504,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
       mbar_arrive_expect_tx(bar(T::BAR_Q), p.tiles * T::TILE_BYTES);
       for (int t = 0; t < p.tiles; ++t)
         for (int b = 0; b < T::NBOX; ++b)
-          tma_load_3d(sbase + T::OFF_Q + t * T::TILE_BYTES + b * T::BOX_BYTES, &tmQ, bar(T::BAR_Q), 64 * b,
+          tma_load_3d(sbase + T::OFF_Q + t * T::TILE_BYTES + b * T::BOX_BYTES, &tmQ, bar(T::BAR_Q), T::BOX_COLS * b,
                       q0 + 128 * t, bh);
       const int total_loads = 2 * n_kv;
       bool ok = true;
@@ -474,7 +516,7 @@ __global__ void __launch_bounds__(FwdTraits<D>::THREADS, 1)
         const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
         for (int b = 0; b < T::NBOX; ++b)
           tma_load_3d(sbase + T::OFF_KV + s * T::TILE_BYTES + b * T::BOX_BYTES, map, bar(T::BAR_KV_FULL + s),
-                      64 * b, 128 * (idx >> 1), bh);
+                      T::BOX_COLS * b, 128 * (idx >> 1), bh);
         issued = idx + 1;
       }
       if (!ok) {

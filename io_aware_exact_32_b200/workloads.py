@@ -14,6 +14,10 @@ Input recipe (all draws on the CPU with ``torch.Generator().manual_seed``):
 * decode: q [B, H, 1, d], K/V caches [B, H, Lmax, d] iid N(0, 1) in bf16 and
   per-sequence lengths L_b drawn uniformly from {lmin, ..., Lmax}; cache slots
   at or beyond L_b hold random data that the kernels must never read.
+* FP8 incoherent processing: the random signs s of M = diag(s) H_d / sqrt(d)
+  are d independent fair +-1 draws (float32).  "Outlier" inputs scale a few
+  whole channels (columns) of Q and K by a power of two after the bf16
+  rounding, the situation the rotation is meant for.
 """
 from __future__ import annotations
 
@@ -32,6 +36,8 @@ __all__ = [
     "DECODE",
     "make_attention_inputs",
     "make_decode_inputs",
+    "make_hadamard_signs",
+    "add_outlier_channels",
     "flops_forward",
     "flops_backward",
     "decode_bytes",
@@ -145,3 +151,16 @@ def decode_bytes(seqlens, H: int, d: int, elem_bytes: int = 2) -> int:
     total_l = int(torch.as_tensor(seqlens).to(torch.int64).sum())
     B = int(torch.as_tensor(seqlens).numel())
     return total_l * H * d * elem_bytes * 2 + 2 * B * H * d * elem_bytes
+
+
+def make_hadamard_signs(d: int, seed: int) -> torch.Tensor:
+    """d independent fair +-1 draws, float32 (the random diagonal of the incoherent-processing matrix)."""
+    gen = torch.Generator().manual_seed(seed)
+    return (torch.randint(0, 2, (d,), generator=gen, dtype=torch.int64) * 2 - 1).to(torch.float32)
+
+
+def add_outlier_channels(x: torch.Tensor, channels, factor: float = 16.0) -> torch.Tensor:
+    """Copy of x [..., d] with the given channels multiplied by ``factor`` (a power of two: exact in bf16)."""
+    y = x.clone()
+    y[..., list(channels)] = y[..., list(channels)] * factor
+    return y

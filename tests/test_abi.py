@@ -26,7 +26,7 @@ def L():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_decode_splitkv", "fa_decode_workspace_size",
-              "fa_get_device_error", "fa_status_string", "fa_version"):
+              "fa_quantize_fp8", "fa_fwd_fp8", "fa_get_device_error", "fa_status_string", "fa_version"):
         assert n in names
 
 
@@ -121,3 +121,30 @@ def test_binding_rejects_bad_tensors():
     q = torch.zeros(1, 1, 4, 64, dtype=torch.float32)
     with pytest.raises(TypeError):
         fa.fa_fwd(q, q, q, q, torch.zeros(1, 1, 4), causal=False)
+
+
+def test_fp8_validation(L):
+    def fwd8(d=128, q=A16, dq=A16, dv=A16, o=A16, Nq=128, Nk=128, B=1):
+        return L.fa_fwd_fp8(q, A16, A16, dq, A16, dv, o, A16, B, 1, Nq, Nk, d, 0.088, 1, NULL)
+
+    assert fwd8(d=64) == 2
+    assert fwd8(d=96) == 2
+    assert fwd8(q=NULL) == 1
+    assert fwd8(dq=NULL) == 1
+    assert fwd8(dv=NULL) == 1
+    assert fwd8(o=MIS) == 3
+    assert fwd8(dq=ctypes.c_void_p(0x10002)) == 3
+    assert fwd8(B=0) == 0
+    assert fwd8(Nq=0, q=NULL, o=NULL) == 0
+
+    def quant(d=128, x=A16, x8=A16, ds=A16, signs=NULL, N=64, B=1):
+        return L.fa_quantize_fp8(x, signs, x8, ds, B, 1, N, d, 1, NULL)
+
+    assert quant(d=32) == 2
+    assert quant(N=-1) == 1
+    assert quant(ds=NULL) == 1
+    assert quant(x=NULL) == 1
+    assert quant(x8=MIS) == 3
+    assert quant(ds=ctypes.c_void_p(0x10001)) == 3
+    assert quant(signs=ctypes.c_void_p(0x10002)) == 3
+    assert quant(B=0) == 0
