@@ -82,6 +82,42 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
                  void* stream);
 
 /*
+ * Additive bias and dropout: O = dropout(softmax(scale * Q K^T + bias
+ * [+ causal mask])) V, the manual path of "优化的注意力实现 (FlashAttention)",
+ * section 优势与集成 (attn_bias added to the scaled scores, dropout on the
+ * weights), and its backward ("FlashAttention 的基本原理", section 2.4 反向传播:
+ * the algorithm covers masking and dropout).
+ *
+ *   bias   [bias_B, bias_H, Nq, Nk] bf16 or NULL; bias_B in {1, B} and
+ *          bias_H in {1, H} (size 1 = broadcast).  -inf masks an entry;
+ *          +inf and NaN are not allowed.  Requires Nk % 8 == 0
+ *          (FA_ERR_UNSUPPORTED otherwise) and a 16-byte aligned pointer.
+ *          The bias is a constant: no gradient is computed for it.
+ *   dropout_p in [0, 1): each weight is dropped with probability
+ *          p8 / 256, p8 = round(256 p) (at most 255), and kept weights are
+ *          scaled by 256 / (256 - p8).  LSE is that of the weights before
+ *          dropout.
+ *   seed, offset: the dropout decisions are regenerated, not stored:
+ *          Philox4x32-10 (Salmon et al., SC 2011) with key (seed low 32
+ *          bits, seed high 32 bits) and counter (key / 4, query / 4,
+ *          b * H + h, offset); byte (key % 4) of output word (query % 4) is
+ *          the entry's random byte u, kept iff u >= p8.  fa_bwd_ext must get
+ *          the same bias, dropout_p, seed and offset as the forward.
+ * Other arguments, layouts and limits as fa_fwd / fa_bwd (same workspace).
+ * dropout_p = 0 and bias = NULL give fa_fwd / fa_bwd's results through the
+ * slower extended kernels.  There is no deterministic variant.
+ */
+FA_API fa_status fa_fwd_ext(const void* q, const void* k, const void* v, const void* bias,
+                 int bias_B, int bias_H, void* o, float* lse, int B, int H, int Nq, int Nk,
+                 int d, float scale, int causal, float dropout_p, unsigned long long seed,
+                 unsigned int offset, void* stream);
+FA_API fa_status fa_bwd_ext(const void* q, const void* k, const void* v, const void* o,
+                 const void* dO, const float* lse, const void* bias, int bias_B, int bias_H,
+                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                 int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                 float dropout_p, unsigned long long seed, unsigned int offset, void* stream);
+
+/*
  * FP8 (E4M3) operands with incoherent processing ("FlashAttention 系列技术详解",
  * section 具体技术, FlashAttention-3): the score and output GEMMs run on FP8
  * tensor cores, and Q and K are first multiplied by a random orthogonal matrix,

@@ -8,8 +8,8 @@ and raises on a non-zero status.  PyTorch provides device memory and streams.
 C-ABI mirrors (same names, torch tensors in place of pointers):
     fa_fwd, fa_bwd, fa_bwd_deterministic, fa_bwd_workspace_size, fa_decode_splitkv, fa_decode_num_splits,
     fa_decode_partials, fa_decode_merge,
-    fa_decode_workspace_size, fa_decode_splitkv_noalloc, fa_quantize_fp8, fa_fwd_fp8,
-    fa_get_device_error, fa_status_string, fa_version
+    fa_decode_workspace_size, fa_decode_splitkv_noalloc, fa_quantize_fp8, fa_fwd_fp8, fa_fwd_ext,
+    fa_bwd_ext, fa_get_device_error, fa_status_string, fa_version
 Convenience wrappers that allocate outputs:
     attention_forward, attention_backward, decode_splitkv, quantize_fp8, attention_forward_fp8
 """
@@ -23,7 +23,8 @@ __all__ = [
     "FAError", "lib", "lib_path",
     "fa_fwd", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size", "fa_decode_splitkv",
     "fa_decode_workspace_size", "fa_decode_num_splits", "fa_decode_partials", "fa_decode_merge",
-    "fa_decode_splitkv_noalloc", "fa_quantize_fp8", "fa_fwd_fp8", "fa_get_device_error", "fa_status_string",
+    "fa_decode_splitkv_noalloc", "fa_quantize_fp8", "fa_fwd_fp8", "fa_fwd_ext", "fa_bwd_ext",
+    "fa_get_device_error", "fa_status_string",
     "fa_version", "attention_forward", "attention_backward", "decode_splitkv", "quantize_fp8",
     "attention_forward_fp8",
 ]
@@ -78,6 +79,12 @@ def lib() -> ctypes.CDLL:
     L.fa_quantize_fp8.restype = i
     L.fa_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     L.fa_fwd_fp8.restype = i
+    u64, u32 = ctypes.c_ulonglong, ctypes.c_uint
+    L.fa_fwd_ext.argtypes = [vp, vp, vp, vp, i, i, vp, vp, i, i, i, i, i, f, i, f, u64, u32, vp]
+    L.fa_fwd_ext.restype = i
+    L.fa_bwd_ext.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, f, u64, u32,
+                             vp]
+    L.fa_bwd_ext.restype = i
     L.fa_get_device_error.argtypes = [vp]
     L.fa_get_device_error.restype = i
     L.fa_status_string.argtypes = [i]
@@ -265,6 +272,56 @@ def fa_decode_merge(part_o, part_ml, o, lse=None, stream=None) -> None:
         _need(lse, "lse", torch.float32, dev, (B, H))
     _check(lib().fa_decode_merge(_ptr(part_o), _ptr(part_ml), R, S, _ptr(o), _ptr(lse), B, H, d,
                                  _stream_ptr(stream)), "fa_decode_merge")
+
+
+def _bias_dims(bias, B, H, Nq, Nk, device):
+    import torch
+    if bias is None:
+        return 1, 1
+    _need(bias, "bias", torch.bfloat16, device)
+    if bias.dim() != 4 or tuple(bias.shape[2:]) != (Nq, Nk) or bias.shape[0] not in (1, B) or \
+            bias.shape[1] not in (1, H):
+        raise ValueError(f"bias has shape {tuple(bias.shape)}, expected [1 or {B}, 1 or {H}, {Nq}, {Nk}]")
+    return int(bias.shape[0]), int(bias.shape[1])
+
+
+def fa_fwd_ext(q, k, v, o, lse, bias=None, causal: bool = False, scale=None, dropout_p: float = 0.0, seed: int = 0,
+               offset: int = 0, stream=None) -> None:
+    """Forward with an additive bias and dropout (see include/fa.h: fa_fwd_ext).  bias [1|B, 1|H, Nq, Nk] bf16
+    or None."""
+    import torch
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    _need(k, "k", torch.bfloat16, dev, (B, H, Nk, d))
+    _need(v, "v", torch.bfloat16, dev, (B, H, Nk, d))
+    _need(o, "o", torch.bfloat16, dev, (B, H, Nq, d))
+    _need(lse, "lse", torch.float32, dev, (B, H, Nq))
+    bB, bH = _bias_dims(bias, B, H, Nq, Nk, dev)
+    _check(lib().fa_fwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), bB, bH, _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                            _scale(scale, d), int(bool(causal)), float(dropout_p), int(seed) & (2 ** 64 - 1),
+                            int(offset) & 0xFFFFFFFF, _stream_ptr(stream)), "fa_fwd_ext")
+
+
+def fa_bwd_ext(q, k, v, o, dO, lse, dq, dk, dv, workspace, bias=None, causal: bool = False, scale=None,
+               dropout_p: float = 0.0, seed: int = 0, offset: int = 0, stream=None) -> None:
+    """Backward of fa_fwd_ext with the same bias, dropout_p, seed and offset (see include/fa.h: fa_bwd_ext)."""
+    import torch
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    dev = q.device
+    for t, n, shp in ((q, "q", (B, H, Nq, d)), (o, "o", (B, H, Nq, d)), (dO, "dO", (B, H, Nq, d)),
+                      (dq, "dq", (B, H, Nq, d)), (k, "k", (B, H, Nk, d)), (v, "v", (B, H, Nk, d)),
+                      (dk, "dk", (B, H, Nk, d)), (dv, "dv", (B, H, Nk, d))):
+        _need(t, n, torch.bfloat16, dev, shp)
+    _need(lse, "lse", torch.float32, dev, (B, H, Nq))
+    _need(workspace, "workspace", torch.uint8, dev)
+    bB, bH = _bias_dims(bias, B, H, Nq, Nk, dev)
+    _check(lib().fa_bwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(bias), bB, bH, _ptr(dq),
+                            _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), B, H, Nq, Nk, d, _scale(scale, d),
+                            int(bool(causal)), float(dropout_p), int(seed) & (2 ** 64 - 1), int(offset) & 0xFFFFFFFF,
+                            _stream_ptr(stream)), "fa_bwd_ext")
 
 
 def _need_e4m3(t, name, device, shape=None):

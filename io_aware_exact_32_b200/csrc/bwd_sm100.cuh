@@ -36,7 +36,7 @@
 
 #include <type_traits>
 
-#include "sm100_ptx.cuh"
+#include "dropout_sm100.cuh"
 
 namespace fa {
 
@@ -111,6 +111,11 @@ struct BwdParams {
   int hgroup;         // heads per scheduling group (1 <= hgroup <= BH)
   float scale, scale_log2;
   int causal;
+  // Bias and dropout instantiation only (as in FwdParams).
+  const __nv_bfloat16* bias;
+  long long bias_sb, bias_sh;
+  int H;
+  DropoutCfg drop;
 };
 
 // ---------------------------------------------------------------------------------------------
@@ -179,7 +184,9 @@ __device__ __forceinline__ void bwd_issue_ss_kmajor(uint32_t tmem_d, uint32_t a_
 
 
 // DQ = false (the deterministic backward): dK and dV only; dQ comes from fa_bwd_dq_kernel.
-template <int D, bool DQ = true>
+// EXT: the forward had an additive bias (p.bias) and dropout (p.drop): P is recomputed with the
+// bias, dV uses the dropped and rescaled weights P o Z, and dS = P o (dP o Z - D).
+template <int D, bool DQ = true, bool EXT = false>
 __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -256,6 +263,11 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     // Query column c of block i sees this key iff c >= cmin (bottom-right causal alignment).
     const int shift = key - (p.Nk - p.Nq);
     const uint32_t ds_row = sbase + T::OFF_DS + r * 128;
+    // EXT: this key's column of the bias (element (q, key) at bias_col[q * Nk]).
+    const __nv_bfloat16* bias_col = nullptr;
+    if constexpr (EXT) {
+      if (p.bias != nullptr && key_ok) bias_col = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + key;
+    }
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
       const int q0 = (i0 + it) * 128;
@@ -266,7 +278,10 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
         const int q = q0 + r;
         const bool in = q < p.Nq;
         const size_t gi = (size_t)bh * p.Nq + (in ? q : 0);
-        const float nlse2 = in ? -p.lse[gi] * kLog2e : -INFINITY;
+        float nlse2 = in ? -p.lse[gi] * kLog2e : -INFINITY;
+        // EXT: a row the bias hides entirely has LSE = -inf; keep its weights at 0 (a -inf bias
+        // entry plus +inf would be NaN).
+        if constexpr (EXT) nlse2 = (nlse2 == INFINITY) ? -INFINITY : nlse2;
         const float nd = in ? -p.dvec[gi] : 0.f;
         asm volatile("bar.sync 1, %0;" ::"n"(128 * T::NCWG) : "memory");
         if (wg == 0) {
@@ -298,11 +313,40 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb + 16 * (ch + 1), dpv[cur ^ 1]);
         }
         uint32_t pk[8], dk[8];
+        // EXT: bias (log2 units, added to -LSE) and dropout factors of this chunk's 16 query columns.
+        float badd[16];
+        float zf[16];
+        if constexpr (EXT) {
+          const int qc = q0 + cb + 16 * ch;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            badd[e] = 0.f;
+            if (bias_col != nullptr && qc + e < p.Nq) {
+              const unsigned short raw = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)(qc + e) * p.Nk));
+              badd[e] = __uint_as_float((uint32_t)raw << 16) * kLog2e;
+            }
+          }
+          if (p.drop.p8 != 0) {
+            uint32_t keepc[16];
+            dropout_keep_colwise(p.drop, (uint32_t)(qc >> 2), (uint32_t)key, (uint32_t)bh, lane, keepc);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) zf[e] = keepc[e] ? p.drop.scale : 0.f;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) zf[e] = 1.f;
+          }
+        }
 #pragma unroll
         for (int i = 0; i < 16; i += 4) {
           const int c = cb + 16 * ch + i;
-          const float4 nl = st4[c >> 2];        // broadcast: every lane reads the same address
+          float4 nl = st4[c >> 2];        // broadcast: every lane reads the same address
           const float4 nd = st4[32 + (c >> 2)];
+          if constexpr (EXT) {
+            nl.x += badd[i];
+            nl.y += badd[i + 1];
+            nl.z += badd[i + 2];
+            nl.w += badd[i + 3];
+          }
           const float2 x01 = ffma2(make_float2(__uint_as_float(sv[cur][i]), __uint_as_float(sv[cur][i + 1])), sc2,
                                    make_float2(nl.x, nl.y));
           const float2 x23 = ffma2(make_float2(__uint_as_float(sv[cur][i + 2]), __uint_as_float(sv[cur][i + 3])),
@@ -315,13 +359,29 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
             p23.x = (key_ok && c + 2 >= cmin) ? p23.x : 0.f;
             p23.y = (key_ok && c + 3 >= cmin) ? p23.y : 0.f;
           }
-          const float2 t01 = fadd2(make_float2(__uint_as_float(dpv[cur][i]), __uint_as_float(dpv[cur][i + 1])),
-                                   make_float2(nd.x, nd.y));
-          const float2 t23 = fadd2(make_float2(__uint_as_float(dpv[cur][i + 2]), __uint_as_float(dpv[cur][i + 3])),
-                                   make_float2(nd.z, nd.w));
+          float2 t01, t23;
+          if constexpr (EXT) {
+            const float2 z01 = make_float2(zf[i], zf[i + 1]), z23 = make_float2(zf[i + 2], zf[i + 3]);
+            t01 = ffma2(make_float2(__uint_as_float(dpv[cur][i]), __uint_as_float(dpv[cur][i + 1])), z01,
+                        make_float2(nd.x, nd.y));
+            t23 = ffma2(make_float2(__uint_as_float(dpv[cur][i + 2]), __uint_as_float(dpv[cur][i + 3])), z23,
+                        make_float2(nd.z, nd.w));
+          } else {
+            t01 = fadd2(make_float2(__uint_as_float(dpv[cur][i]), __uint_as_float(dpv[cur][i + 1])),
+                        make_float2(nd.x, nd.y));
+            t23 = fadd2(make_float2(__uint_as_float(dpv[cur][i + 2]), __uint_as_float(dpv[cur][i + 3])),
+                        make_float2(nd.z, nd.w));
+          }
           const float2 d01 = fmul2(p01, t01), d23 = fmul2(p23, t23);
-          pk[i / 2] = pack_bf16x2(p01.x, p01.y);
-          pk[i / 2 + 1] = pack_bf16x2(p23.x, p23.y);
+          if constexpr (EXT) {
+            const float2 pz01 = fmul2(p01, make_float2(zf[i], zf[i + 1]));
+            const float2 pz23 = fmul2(p23, make_float2(zf[i + 2], zf[i + 3]));
+            pk[i / 2] = pack_bf16x2(pz01.x, pz01.y);
+            pk[i / 2 + 1] = pack_bf16x2(pz23.x, pz23.y);
+          } else {
+            pk[i / 2] = pack_bf16x2(p01.x, p01.y);
+            pk[i / 2 + 1] = pack_bf16x2(p23.x, p23.y);
+          }
           dk[i / 2] = pack_bf16x2(d01.x, d01.y);
           dk[i / 2 + 1] = pack_bf16x2(d23.x, d23.y);
         }

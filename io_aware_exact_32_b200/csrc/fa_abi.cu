@@ -123,17 +123,58 @@ int decode_chunk(int Lmax, int S) {
   return (c + 31) & ~31;
 }
 
-template <int D, bool F8 = false>
+// Bias and dropout of the *_ext calls, validated on the host.
+struct ExtArgs {
+  const __nv_bfloat16* bias;  // null: no bias
+  long long sb, sh;           // element strides of b and h in the bias (0 where broadcast)
+  int H;
+  fa::DropoutCfg drop;
+};
+
+template <typename P>
+void set_ext(P& p, const ExtArgs* ext) {
+  p.bias = ext ? ext->bias : nullptr;
+  p.bias_sb = ext ? ext->sb : 0;
+  p.bias_sh = ext ? ext->sh : 0;
+  p.H = ext ? ext->H : 1;
+  p.drop = ext ? ext->drop : fa::DropoutCfg{0u, 1.f, 0u, 0u, 0u};
+}
+
+// Checks the bias shape and dropout probability and fills ext.
+fa_status make_ext(ExtArgs* ext, const void* bias, int bias_B, int bias_H, int B, int H, int Nq, int Nk,
+                   float dropout_p, unsigned long long seed, unsigned int offset) {
+  if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_INVALID_ARG;
+  long r = std::lround(256.0 * (double)dropout_p);
+  const uint32_t p8 = (uint32_t)(r > 255 ? 255 : r);
+  ext->drop = fa::DropoutCfg{p8, (float)(256.0 / (256.0 - (double)p8)), (uint32_t)(seed & 0xffffffffull),
+                             (uint32_t)(seed >> 32), offset};
+  ext->H = H;
+  ext->bias = static_cast<const __nv_bfloat16*>(bias);
+  ext->sb = ext->sh = 0;
+  if (bias) {
+    if ((bias_B != 1 && bias_B != B) || (bias_H != 1 && bias_H != H)) return FA_ERR_INVALID_ARG;
+    if (Nk % 8 != 0) return FA_ERR_UNSUPPORTED;  // bias rows are read in 16-byte chunks
+    if (!aligned16(bias)) return FA_ERR_MISALIGNED;
+    const long long plane = (long long)Nq * Nk;
+    ext->sh = bias_H == 1 ? 0 : plane;
+    ext->sb = bias_B == 1 ? 0 : (long long)bias_H * plane;
+  }
+  return FA_OK;
+}
+
+template <int D, bool F8 = false, bool EXT = false>
 fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int BH, int Nq, int Nk,
                      float scale, int causal, cudaStream_t stream, const float* descale_q = nullptr,
-                     const float* descale_k = nullptr, const float* descale_v = nullptr) {
+                     const float* descale_k = nullptr, const float* descale_v = nullptr,
+                     const ExtArgs* ext = nullptr) {
   using T = fa::FwdTraits<D, F8>;
   CUtensorMap mq, mk, mv;
   if (!make_map_3d(&mq, q, D, Nq, BH, F8) || !make_map_3d(&mk, k, D, Nk, BH, F8) ||
       !make_map_3d(&mv, v, D, Nk, BH, F8))
     return FA_ERR_CUDA;
-  if (!set_smem(fa::fa_fwd_kernel<D, F8>, T::SMEM_BYTES)) return FA_ERR_CUDA;
+  if (!set_smem(fa::fa_fwd_kernel<D, F8, EXT>, T::SMEM_BYTES)) return FA_ERR_CUDA;
   fa::FwdParams p;
+  set_ext(p, ext);
   p.descale_q = descale_q;
   p.descale_k = descale_k;
   p.descale_v = descale_v;
@@ -149,7 +190,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   p.causal = causal ? 1 : 0;
   const long long blocks = (long long)p.nunits * BH;
   if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  fa::fa_fwd_kernel<D, F8><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  fa::fa_fwd_kernel<D, F8, EXT><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -159,7 +200,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
 template <int D>
 fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                      void* dq, void* dk, void* dv, void* ws, int BH, int Nq, int Nk, float scale, int causal,
-                     cudaStream_t stream, bool deterministic) {
+                     cudaStream_t stream, bool deterministic, const ExtArgs* ext = nullptr) {
   if (Nk == 0) deterministic = false;
   using T = fa::BwdTraits<D>;
   const long long rows = (long long)BH * Nq;
@@ -177,9 +218,11 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
         !make_map_3d(&mdo, dO, D, Nq, BH) || !make_map_3d_f32(&mdq, dq_acc, D, Nq > 0 ? Nq : 1, BH))
       return FA_ERR_CUDA;
     if (!set_smem(fa::fa_bwd_main_kernel<D, true>, T::SMEM_BYTES) ||
-        !set_smem(fa::fa_bwd_main_kernel<D, false>, T::SMEM_BYTES))
+        !set_smem(fa::fa_bwd_main_kernel<D, false>, T::SMEM_BYTES) ||
+        (ext && !set_smem(fa::fa_bwd_main_kernel<D, true, true>, T::SMEM_BYTES)))
       return FA_ERR_CUDA;
     fa::BwdParams p;
+    set_ext(p, ext);
     p.lse = lse;
     p.dvec = dvec;
     p.dq_acc = dq_acc;
@@ -202,7 +245,10 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.causal = causal ? 1 : 0;
     const long long blocks = (long long)p.nkt * BH;
     if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-    if (deterministic)
+    if (ext)
+      fa::fa_bwd_main_kernel<D, true, true><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
+                                                                                                     mdq, p);
+    else if (deterministic)
       fa::fa_bwd_main_kernel<D, false><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
     else
       fa::fa_bwd_main_kernel<D, true><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
@@ -382,7 +428,7 @@ size_t fa_bwd_workspace_size(int B, int H, int Nq, int d) {
 
 static fa_status bwd_entry(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                  void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H, int Nq, int Nk, int d,
-                 float scale, int causal, void* stream, bool deterministic) {
+                 float scale, int causal, void* stream, bool deterministic, const ExtArgs* ext = nullptr) {
   fa_status st = check_common(B, H, Nq, Nk, d, scale);
   if (st != FA_OK) return st;
   const long long BH = (long long)B * H;
@@ -397,9 +443,48 @@ static fa_status bwd_entry(const void* q, const void* k, const void* v, const vo
   if (need > 0 && (!workspace || ws_bytes < need)) return FA_ERR_WORKSPACE;
   if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s, deterministic)
+  return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s, deterministic,
+                                  ext)
                  : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s,
-                                   deterministic);
+                                   deterministic, ext);
+}
+
+fa_status fa_fwd_ext(const void* q, const void* k, const void* v, const void* bias, int bias_B, int bias_H, void* o,
+                     float* lse, int B, int H, int Nq, int Nk, int d, float scale, int causal, float dropout_p,
+                     unsigned long long seed, unsigned int offset, void* stream) {
+  fa_status st = check_common(B, H, Nq, Nk, d, scale);
+  if (st != FA_OK) return st;
+  ExtArgs ext;
+  if ((st = make_ext(&ext, bias, bias_B, bias_H, B, H, Nq, Nk, dropout_p, seed, offset)) != FA_OK) return st;
+  const long long BH = (long long)B * H;
+  if (BH == 0 || Nq == 0) return FA_OK;
+  if (!q || !o || !lse || (Nk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse) || (Nk > 0 && (!aligned16(k) || !aligned16(v))))
+    return FA_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (Nk == 0) {
+    const long long rows = BH * Nq;
+    const long long n = rows * d;
+    fa::fa_fwd_empty_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(static_cast<__nv_bfloat16*>(o), lse, rows,
+                                                                         d);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  }
+  return d == 64 ? launch_fwd<64, false, true>(q, k, v, o, lse, (int)BH, Nq, Nk, scale, causal, s, nullptr, nullptr,
+                                               nullptr, &ext)
+                 : launch_fwd<128, false, true>(q, k, v, o, lse, (int)BH, Nq, Nk, scale, causal, s, nullptr, nullptr,
+                                                nullptr, &ext);
+}
+
+fa_status fa_bwd_ext(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                     const void* bias, int bias_B, int bias_H, void* dq, void* dk, void* dv, void* workspace,
+                     size_t ws_bytes, int B, int H, int Nq, int Nk, int d, float scale, int causal, float dropout_p,
+                     unsigned long long seed, unsigned int offset, void* stream) {
+  fa_status st = check_common(B, H, Nq, Nk, d, scale);
+  if (st != FA_OK) return st;
+  ExtArgs ext;
+  if ((st = make_ext(&ext, bias, bias_B, bias_H, B, H, Nq, Nk, dropout_p, seed, offset)) != FA_OK) return st;
+  return bwd_entry(q, k, v, o, dO, lse, dq, dk, dv, workspace, ws_bytes, B, H, Nq, Nk, d, scale, causal, stream,
+                   false, &ext);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,

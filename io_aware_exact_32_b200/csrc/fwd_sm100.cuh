@@ -28,7 +28,7 @@
 //    by the sum of those rounded weights, LSE by the exact fp32 sum.
 #pragma once
 
-#include "sm100_ptx.cuh"
+#include "dropout_sm100.cuh"
 
 namespace fa {
 
@@ -92,6 +92,12 @@ struct FwdParams {
   const float* descale_q;
   const float* descale_k;
   const float* descale_v;
+  // Bias and dropout instantiation only.  bias: [Bb, Hb, Nq, Nk] bf16 or null, b / h element
+  // strides bias_sb / bias_sh (0 where broadcast); H splits the (batch, head) index.
+  const __nv_bfloat16* bias;
+  long long bias_sb, bias_sh;
+  int H;
+  DropoutCfg drop;
 };
 
 // Number of 128-key tiles the CTA owning query rows [q0, q0 + span) must visit.
@@ -157,10 +163,36 @@ __device__ __forceinline__ float max64(const float* s) {
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-template <int D, bool F8 = false>
+// Bias step of the EXT forward for 64 keys [k0, k0 + 64) of one row: s <- s * scale_log2 + bias * log2(e)
+// (a key past Nk reads no bias; it is already -inf).  Rows are read as 16-byte chunks, so Nk is a
+// multiple of 8 whenever a bias is given.
+__device__ __forceinline__ void fwd_apply_bias(float* s, const __nv_bfloat16* bias_row, int k0, int Nk,
+                                               float scale_log2) {
+  constexpr float kLog2eF = 1.4426950408889634f;
+  if (bias_row == nullptr) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) s[c] *= scale_log2;
+    return;
+  }
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (k0 + 8 * g < Nk) raw = __ldg(reinterpret_cast<const uint4*>(bias_row + k0 + 8 * g));
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      s[8 * g + 2 * i] = fmaf(s[8 * g + 2 * i], scale_log2, bf16lo_to_f32(w[i]) * kLog2eF);
+      s[8 * g + 2 * i + 1] = fmaf(s[8 * g + 2 * i + 1], scale_log2, bf16hi_to_f32(w[i]) * kLog2eF);
+    }
+  }
+}
+
+// EXT: the scores get an additive bias (p.bias) and the weights dropout (p.drop) before P V.
+template <int D, bool F8 = false, bool EXT = false>
 __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  static_assert(!(F8 && EXT), "bias and dropout are not combined with FP8 operands");
   using T = FwdTraits<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -223,7 +255,14 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
     float m_run = -INFINITY, l_run = 0.f, lr_run = 0.f;
     float scale_log2 = p.scale_log2;
     if constexpr (F8) scale_log2 *= __ldg(p.descale_q + bh) * __ldg(p.descale_k + bh);
-    const float2 sc2 = make_float2(scale_log2, scale_log2);
+    // EXT: the scores are turned into log2-domain logits s * scale * log2(e) + bias * log2(e) in
+    // place, so the exponent step below multiplies by 1.
+    const float2 sc2 = EXT ? make_float2(1.f, 1.f) : make_float2(scale_log2, scale_log2);
+    const __nv_bfloat16* bias_row = nullptr;
+    if constexpr (EXT) {
+      if (p.bias != nullptr && row < p.Nq)
+        bias_row = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + (size_t)row * p.Nk;
+    }
     bool ok = true;
     for (int step = 0; step < n_own; ++step) {
       const int j = two ? step : 2 * step + t;  // key tile
@@ -244,6 +283,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
         for (int c = 0; c < 64; ++c)
           if (c > lim) s[c] = -INFINITY;
       }
+      if constexpr (EXT) fwd_apply_bias(s, bias_row, 128 * j, p.Nk, scale_log2);
       const float mx_a = max64(s);
       tmem_wait_ld_x64(sb);
       if (masked) {
@@ -251,8 +291,9 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
         for (int c = 0; c < 64; ++c)
           if (c + 64 > lim) s2[c] = -INFINITY;
       }
+      if constexpr (EXT) fwd_apply_bias(s2, bias_row, 128 * j + 64, p.Nk, scale_log2);
       const float mx = fmaxf(mx_a, max64(s2));
-      const float m_tile = mx * scale_log2;
+      const float m_tile = EXT ? mx : mx * scale_log2;
       float alpha = 1.f;
       bool resc = false;
       if (m_tile > m_run + kRescaleThreshold) {
@@ -294,6 +335,11 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
         for (int ch = 0; ch < 4; ++ch) {
           const float* src = (ch < 2) ? s + 32 * ch : s2 + 32 * (ch - 2);
           uint32_t pk[16];
+          uint32_t keep[8];  // EXT with dropout: 0xff per kept key of this chunk's 8 key quads
+          if constexpr (EXT) {
+            if (p.drop.p8 != 0) dropout_keep_rowwise(p.drop, (uint32_t)(32 * j + 8 * ch), (uint32_t)row, (uint32_t)bh,
+                                                     lane, keep);
+          }
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const float2 x = ffma2(make_float2(src[2 * c], src[2 * c + 1]), sc2, nb2);
@@ -306,6 +352,10 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
             pk[c] = pack_bf16x2(e.x, e.y);
             sum_e[c & 1] = fadd2(sum_e[c & 1], e);
             sum_r[c & 1] = fadd2(sum_r[c & 1], make_float2(bf16lo_to_f32(pk[c]), bf16hi_to_f32(pk[c])));
+            if constexpr (EXT) {
+              // Dropped weights leave the normalising sums untouched and enter P V as +0.
+              if (p.drop.p8 != 0) pk[c] &= __byte_perm(keep[c >> 1], 0u, (c & 1) ? 0x3322u : 0x1100u);
+            }
           }
           tmem_st32x32b_x16(lane_addr + colS + 16 * ch, pk);
         }
@@ -367,6 +417,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
       tc_fence_after();
       float num = 1.f;
       if constexpr (F8) num = __ldg(p.descale_v + bh);
+      if constexpr (EXT) num = p.drop.scale;
       const float inv = lr_run > 0.f ? num / lr_run : 0.f;
       const bool in_range = row < p.Nq;
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D;

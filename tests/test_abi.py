@@ -26,7 +26,8 @@ def L():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_decode_splitkv", "fa_decode_workspace_size",
-              "fa_quantize_fp8", "fa_fwd_fp8", "fa_get_device_error", "fa_status_string", "fa_version"):
+              "fa_quantize_fp8", "fa_fwd_fp8", "fa_fwd_ext", "fa_bwd_ext", "fa_get_device_error", "fa_status_string",
+              "fa_version"):
         assert n in names
 
 
@@ -148,3 +149,26 @@ def test_fp8_validation(L):
     assert quant(ds=ctypes.c_void_p(0x10001)) == 3
     assert quant(signs=ctypes.c_void_p(0x10002)) == 3
     assert quant(B=0) == 0
+
+
+def test_ext_validation(L):
+    def fwdx(p=0.1, bias=A16, bB=1, bH=1, Nk=128, B=2, d=64):
+        return L.fa_fwd_ext(A16, A16, A16, bias, bB, bH, A16, A16, B, 2, 128, Nk, d, 0.125, 1, p, 7, 0, NULL)
+
+    assert fwdx(p=1.0) == 1
+    assert fwdx(p=-0.1) == 1
+    assert fwdx(p=float("nan")) == 1
+    assert fwdx(Nk=130) == 2            # a bias needs Nk % 8 == 0
+    assert fwdx(bB=3) == 1
+    assert fwdx(bH=0) == 1
+    assert fwdx(bias=ctypes.c_void_p(0x10008)) == 3
+    assert fwdx(d=96) == 2
+    assert fwdx(B=0) == 0
+
+    def bwdx(p=0.1, bias=A16, ws=A16):
+        args = [A16] * 6 + [bias, 1, 1] + [A16] * 3
+        return L.fa_bwd_ext(*args, ws, 1 << 30, 1, 1, 128, 128, 64, 0.125, 0, p, 7, 0, NULL)
+
+    assert bwdx(p=1.5) == 1
+    assert bwdx(bias=ctypes.c_void_p(0x10004)) == 3
+    assert bwdx(ws=NULL) == 4
