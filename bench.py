@@ -544,6 +544,19 @@ def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
             "fwd_incl_quantize_tflops": ff / (t_f8 + t_q8) / 1e12}
         del q8, k8, v8, dsq, dsk, dsv, o8, lse8
         if n == 4096:
+            # Bias (one [Nq, Nk] plane per head, broadcast over the batch) and dropout p = 0.1.
+            gb = torch.Generator().manual_seed(9)
+            bias = (torch.randn(1, cfg.H, cfg.Nq, cfg.Nk, generator=gb) * 0.5).to(torch.bfloat16).to(dev)
+            oe, lsee = torch.empty_like(o), torch.empty_like(lse)
+            t_fe = timed(lambda: fa.fa_fwd_ext(q, k, v, oe, lsee, bias, True, cfg.scale, 0.1, 1234, 0, stream))
+            t_be = timed(lambda: fa.fa_bwd_ext(q, k, v, oe, do, lsee, dq, dk, dv, ws, bias, True, cfg.scale, 0.1, 1234,
+                                               0, stream))
+            res["bias_dropout_causal_n4096_d128"] = {
+                "fwd_tflops": ff / t_fe / 1e12, "bwd_tflops": fb / t_be / 1e12,
+                "fwd_bwd_tflops": (ff + fb) / (t_fe + t_be) / 1e12, "fwd_ms": 1e3 * t_fe, "bwd_ms": 1e3 * t_be,
+                "vs_plain_fwd": t_f / t_fe, "vs_plain_bwd": t_b / t_be,
+                "note": "bias [1, H, N, N] bf16 (read once per query tile), dropout p = 0.1"}
+            del bias, oe, lsee
             t_bd = timed(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, True, cfg.scale, stream,
                                            deterministic=True))
             res["deterministic_bwd_causal_n4096_d128"] = {"bwd_tflops": fb / t_bd / 1e12, "bwd_ms": 1e3 * t_bd,
@@ -564,7 +577,8 @@ def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
     return res
 
 
-CASES = ("fwd_c2", "bwd_c2", "fwd_n4096_d128", "bwd_n4096_d128", "fwd_fp8_n4096_d128", "decode")
+CASES = ("fwd_c2", "bwd_c2", "fwd_n4096_d128", "bwd_n4096_d128", "fwd_fp8_n4096_d128", "fwd_ext_n4096_d128",
+         "bwd_ext_n4096_d128", "decode")
 
 
 def run_case(args):
@@ -601,6 +615,19 @@ def run_case(args):
             v8, dsv = fa.quantize_fp8(v, None, False, stream)
             fn = lambda: fa.fa_fwd_fp8(q8, k8, v8, dsq, dsk, dsv, o, lse, causal, cfg.scale, stream)
             units = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal) / 1e12
+        elif name.endswith("ext_n4096_d128"):
+            gb = torch.Generator().manual_seed(9)
+            bias = (torch.randn(1, cfg.H, cfg.Nq, cfg.Nk, generator=gb) * 0.5).to(torch.bfloat16).to(dev)
+            fa.fa_fwd_ext(q, k, v, o, lse, bias, causal, cfg.scale, 0.1, 1234, 0, stream)
+            if name.startswith("fwd"):
+                fn = lambda: fa.fa_fwd_ext(q, k, v, o, lse, bias, causal, cfg.scale, 0.1, 1234, 0, stream)
+                units = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal) / 1e12
+            else:
+                ws = torch.empty(fa.fa_bwd_workspace_size(cfg.B, cfg.H, cfg.Nq, cfg.d), dtype=torch.uint8, device=dev)
+                dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+                fn = lambda: fa.fa_bwd_ext(q, k, v, o, do, lse, dq, dk, dv, ws, bias, causal, cfg.scale, 0.1, 1234, 0,
+                                           stream)
+                units = W.flops_backward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal) / 1e12
         elif name.startswith("fwd"):
             fn = lambda: fa.fa_fwd(q, k, v, o, lse, causal, cfg.scale, stream)
             units = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal) / 1e12
