@@ -1,6 +1,6 @@
 // Thin inline-PTX wrappers for the sm_100a features the kernels use:
-// mbarriers with bounded waits, TMA (tensor and plain bulk copies, no
-// multicast), and the 5th-generation tensor core (tcgen05: TMEM allocation,
+// mbarriers with bounded waits, TMA (tensor and plain bulk copies, each CTA
+// loading only for itself), and the 5th-generation tensor core (tcgen05: TMEM allocation,
 // MMA with shared-memory / tensor-memory operands, commit, TMEM load/store).
 //
 // Every wait here is bounded by wall-clock time (%globaltimer).  A wait that
