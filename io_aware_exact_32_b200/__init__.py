@@ -125,6 +125,9 @@ def _need(t, name, dtype, device, shape=None):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device.type != "cuda":
+        # The kernels take device pointers: a host tensor must never reach them.
+        raise ValueError(f"{name} must be a CUDA tensor, got {t.device}")
     if t.device != device:
         raise ValueError(f"{name} must be on {device}, got {t.device}")
     if not t.is_contiguous():
@@ -278,10 +281,12 @@ def _bias_dims(bias, B, H, Nq, Nk, device):
     import torch
     if bias is None:
         return 1, 1
-    _need(bias, "bias", torch.bfloat16, device)
+    if not isinstance(bias, torch.Tensor):
+        raise TypeError("bias must be a torch.Tensor")
     if bias.dim() != 4 or tuple(bias.shape[2:]) != (Nq, Nk) or bias.shape[0] not in (1, B) or \
             bias.shape[1] not in (1, H):
         raise ValueError(f"bias has shape {tuple(bias.shape)}, expected [1 or {B}, 1 or {H}, {Nq}, {Nk}]")
+    _need(bias, "bias", torch.bfloat16, device)
     return int(bias.shape[0]), int(bias.shape[1])
 
 

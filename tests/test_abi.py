@@ -172,3 +172,23 @@ def test_ext_validation(L):
     assert bwdx(p=1.5) == 1
     assert bwdx(bias=ctypes.c_void_p(0x10004)) == 3
     assert bwdx(ws=NULL) == 4
+
+
+def test_binding_rejects_host_tensors_and_bad_shapes():
+    """Host tensors never reach the C ABI (its kernels take device pointers), and shape errors of the
+    bias / FP8 arguments are caught in Python."""
+    torch = pytest.importorskip("torch")
+    q = torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16)
+    o = torch.zeros_like(q)
+    lse = torch.zeros(1, 2, 16)
+    for call in (lambda: fa.fa_fwd(q, q, q, o, lse, causal=False),
+                 lambda: fa.fa_fwd_ext(q, q, q, o, lse, None, False),
+                 lambda: fa.quantize_fp8(q, None, True),
+                 lambda: fa.fa_fwd_fp8(q.to(torch.uint8), q.to(torch.uint8), q.to(torch.uint8),
+                                       torch.zeros(1, 2), torch.zeros(1, 2), torch.zeros(1, 2), o, lse, False)):
+        with pytest.raises(ValueError, match="CUDA"):
+            call()
+    with pytest.raises(ValueError, match="bias"):
+        fa._bias_dims(torch.zeros(1, 3, 16, 16, dtype=torch.bfloat16), 1, 2, 16, 16, q.device)
+    with pytest.raises(ValueError, match="bias"):
+        fa._bias_dims(torch.zeros(1, 2, 16, 8, dtype=torch.bfloat16), 1, 2, 16, 16, q.device)
