@@ -483,9 +483,32 @@ def run_ours(args):
     return 0
 
 
+def long_context_measurement(fa, W, dev, stream, peaks, timed, cfg=None):
+    """Causal forward and forward+backward on the long-context case (B=1, H=16, N=65536, d=128, 1% of
+    key rows x8); ``timed(fn)`` returns seconds per call."""
+    import torch
+    c = cfg or W.LONG
+    x = W.make_config_inputs(c)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    del x
+    o, lse = fa.attention_forward(q, k, v, causal=True, scale=c.scale)
+    ws = torch.empty(fa.fa_bwd_workspace_size(c.B, c.H, c.Nq, c.d), dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    t_f = timed(lambda: fa.fa_fwd(q, k, v, o, lse, True, c.scale, stream))
+    t_b = timed(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, True, c.scale, stream))
+    ff = W.flops_forward(c.B, c.H, c.Nq, c.Nk, c.d, True)
+    fb = W.flops_backward(c.B, c.H, c.Nq, c.Nk, c.d, True)
+    f1, f2 = ff / t_f / 1e12, (ff + fb) / (t_f + t_b) / 1e12
+    return {"B": c.B, "H": c.H, "N": c.Nq, "fwd_tflops": f1, "fwd_frac": f1 / peaks["bf16_tflops"],
+            "fwd_frac_of_2250": f1 / 2250.0, "bwd_tflops": fb / t_b / 1e12, "fwd_bwd_tflops": f2,
+            "fwd_bwd_frac": f2 / peaks["bf16_tflops"], "fwd_bwd_frac_of_2250": f2 / 2250.0, "fwd_ms": 1e3 * t_f,
+            "bwd_ms": 1e3 * t_b, "device_status": fa.fa_get_device_error(stream)}
+
+
 def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
     """d=128 causal forward and forward+backward at N = 4096, 8192, 16384 (the sweep's B*N = 16384
-    tokens, H=16), and split-KV decode bandwidth."""
+    tokens, H=16), the FP8 and bias / dropout variants, the deterministic backward, split-KV decode
+    bandwidth, and the 65536-token causal case."""
     import torch
     res = {}
 
@@ -562,6 +585,11 @@ def extra_measurements(fa, W, dev, stream, flush_buf, peaks, iters=10):
             res["deterministic_bwd_causal_n4096_d128"] = {"bwd_tflops": fb / t_bd / 1e12, "bwd_ms": 1e3 * t_bd,
                                                           "vs_default_bwd": t_b / t_bd}
         del q, k, v, do, o, lse, dq, dk, dv, ws, x
+    # Its failure is recorded rather than raised, so that the lines above are still reported.
+    try:
+        res["long_n65536_d128_causal_peaked"] = long_context_measurement(fa, W, dev, stream, peaks, timed)
+    except Exception as e:  # noqa: BLE001 - reported in the JSON line
+        res["long_n65536_d128_causal_peaked"] = {"error": f"{type(e).__name__}: {e}"}
     dc = W.DECODE
     xd = W.make_decode_inputs(dc.B, dc.H, dc.Lmax, dc.d, dc.lmin, dc.seed)
     qd, kc, vc = (xd[n].to(dev) for n in ("q", "k_cache", "v_cache"))

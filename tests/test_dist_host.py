@@ -65,3 +65,30 @@ def test_single_process_defaults(monkeypatch):
 def test_measured_peaks_read():
     p = bench.measured_peaks()
     assert p["bf16_tflops"] > 100 and p["hbm_gbs"] > 1000
+
+
+def test_long_context_measurement_host_logic():
+    """bench.py's long-context block with a stand-in for the library (no GPU call): it allocates the
+    right shapes and turns times into the FLOP-rate fields."""
+    import types
+
+    import torch
+
+    import bench
+    from io_aware_exact_32_b200 import workloads as W
+
+    calls = []
+    fake = types.SimpleNamespace(
+        attention_forward=lambda q, k, v, causal, scale: (torch.empty_like(q), torch.empty(q.shape[:3])),
+        fa_bwd_workspace_size=lambda B, H, N, d: 256,
+        fa_fwd=lambda *a: calls.append("fwd"),
+        fa_bwd=lambda *a: calls.append("bwd"),
+        fa_get_device_error=lambda stream: 0)
+    small = W.AttnConfig("long_small", 1, 2, 256, 256, 128, (True,), seed=3, peaked_frac=0.01)
+    out = bench.long_context_measurement(fake, W, torch.device("cpu"), None, {"bf16_tflops": 1000.0},
+                                         lambda fn: (fn(), 1e-3)[1], cfg=small)
+    assert calls == ["fwd", "bwd"]
+    ff = W.flops_forward(1, 2, 256, 256, 128, True)
+    assert abs(out["fwd_tflops"] - ff / 1e-3 / 1e12) < 1e-12
+    assert abs(out["fwd_bwd_tflops"] - 3.5 * ff / 2e-3 / 1e12) < 1e-12
+    assert out["device_status"] == 0 and out["N"] == 256
