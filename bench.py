@@ -442,7 +442,7 @@ def run_ours(args):
             roofline["traffic_unit"] = "bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)"
 
     extra = {}
-    if not args.no_extra:
+    if not args.no_extra and world == 1:  # single-GPU kernel measurements; the N > 1 line is the headline alone
         extra = extra_measurements(fa, W, dev, stream, flush_buf, peaks)
 
     if world > 1:
