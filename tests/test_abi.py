@@ -192,3 +192,26 @@ def test_binding_rejects_host_tensors_and_bad_shapes():
         fa._bias_dims(torch.zeros(1, 3, 16, 16, dtype=torch.bfloat16), 1, 2, 16, 16, q.device)
     with pytest.raises(ValueError, match="bias"):
         fa._bias_dims(torch.zeros(1, 2, 16, 8, dtype=torch.bfloat16), 1, 2, 16, 16, q.device)
+
+
+def test_binding_argument_counts_match_the_header(L):
+    """Each ctypes signature in the binding has as many arguments as the C declaration in include/fa.h."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(([^)]*)\)\s*;", text)
+    assert len(decls) == len(declared_functions())
+    for name, params in decls:
+        params = params.strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        fn = getattr(L, name)
+        assert fn.argtypes is not None, f"{name}: no argtypes in the binding"
+        assert len(fn.argtypes) == n, f"{name}: binding has {len(fn.argtypes)} arguments, header {n}"
+
+
+def test_product_package_never_imports_the_oracle():
+    pkg = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "io_aware_exact_32_b200")
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".inc")):
+                src = open(os.path.join(root, f), encoding="utf-8").read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", src, flags=re.M), f
+                assert "oracle/" not in src, f
