@@ -94,9 +94,9 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
  *          (FA_ERR_UNSUPPORTED otherwise) and a 16-byte aligned pointer.
  *          The bias is a constant: no gradient is computed for it.
  *   dropout_p in [0, 1): each weight is dropped with probability
- *          p8 / 256, p8 = round(256 p) (at most 255), and kept weights are
- *          scaled by 256 / (256 - p8).  LSE is that of the weights before
- *          dropout.
+ *          p8 / 256, p8 = floor(256 p + 1/2) (at most 255; a tie goes
+ *          up), and kept weights are scaled by 256 / (256 - p8).  LSE is
+ *          that of the weights before dropout.
  *   seed, offset: the dropout decisions are regenerated, not stored:
  *          Philox4x32-10 (Salmon et al., SC 2011) with key (seed low 32
  *          bits, seed high 32 bits) and counter (key / 4, query / 4,
@@ -294,7 +294,9 @@ FA_API fa_status fa_decode_merge(const float* part_o, const float* part_ml, int 
  *
  * The first call on each device looks up that device's address of the scratch
  * array (cudaGetSymbolAddress, with the device current); make that first call
- * before any stream capture.  All calls share the one array: calls whose
+ * before any stream capture.  The address is kept for the life of the
+ * process, so this entry point does not survive a cudaDeviceReset of that
+ * device in the same process.  All calls share the one array: calls whose
  * kernels overlap on the GPU (different streams, no ordering between them)
  * race on it and must be serialised by the caller.  Nothing needs clearing
  * between calls: every partial is written before it is read.
@@ -310,6 +312,20 @@ FA_API fa_status fa_decode_splitkv_noalloc(const void* q, const void* k_cache, c
  * call.  Returns FA_ERR_CUDA if the synchronisation itself failed.
  */
 FA_API fa_status fa_get_device_error(void* stream);
+
+/*
+ * Test hook, not for production use: sets the time after which every pipeline
+ * wait of this library's kernels on the current device gives up (default 2 s;
+ * limit_ns == 0 restores it), and caps the hardware suspend time of those waits
+ * at the same value.  With a limit of a few hundred nanoseconds the waits of a
+ * healthy kernel run out: each CTA records FA_ERR_TIMEOUT, stops, waits (with
+ * the fixed 2 s limit) for its own copies and MMAs still in flight, frees its
+ * tensor memory and returns, so the give-up path can be tested without a
+ * fault.  The setting is per device and lasts until changed; the call is
+ * synchronous (it copies to device constant memory).  Returns FA_ERR_CUDA if
+ * the copy fails.  The pages have no counterpart: this exists for testing.
+ */
+FA_API fa_status fa_debug_set_wait_limit(unsigned long long limit_ns);
 
 /* Static, NUL-terminated description of a status code. */
 FA_API const char* fa_status_string(fa_status status);

@@ -9,7 +9,7 @@ C-ABI mirrors (same names, torch tensors in place of pointers):
     fa_fwd, fa_bwd, fa_bwd_deterministic, fa_bwd_workspace_size, fa_decode_splitkv, fa_decode_num_splits,
     fa_decode_partials, fa_decode_merge,
     fa_decode_workspace_size, fa_decode_splitkv_noalloc, fa_quantize_fp8, fa_fwd_fp8, fa_fwd_ext,
-    fa_bwd_ext, fa_get_device_error, fa_status_string, fa_version
+    fa_bwd_ext, fa_get_device_error, fa_debug_set_wait_limit, fa_status_string, fa_version
 Convenience wrappers that allocate outputs:
     attention_forward, attention_backward, decode_splitkv, quantize_fp8, attention_forward_fp8
 """
@@ -24,7 +24,7 @@ __all__ = [
     "fa_fwd", "fa_bwd", "fa_bwd_deterministic", "fa_bwd_workspace_size", "fa_decode_splitkv",
     "fa_decode_workspace_size", "fa_decode_num_splits", "fa_decode_partials", "fa_decode_merge",
     "fa_decode_splitkv_noalloc", "fa_quantize_fp8", "fa_fwd_fp8", "fa_fwd_ext", "fa_bwd_ext",
-    "fa_get_device_error", "fa_status_string",
+    "fa_get_device_error", "fa_debug_set_wait_limit", "fa_status_string",
     "fa_version", "attention_forward", "attention_backward", "decode_splitkv", "quantize_fp8",
     "attention_forward_fp8",
 ]
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_ext.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, f, u64, u32,
                              vp]
     L.fa_bwd_ext.restype = i
+    L.fa_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+    L.fa_debug_set_wait_limit.restype = i
     L.fa_get_device_error.argtypes = [vp]
     L.fa_get_device_error.restype = i
     L.fa_status_string.argtypes = [i]
@@ -103,11 +105,24 @@ def fa_version() -> int:
     return lib().fa_version()
 
 
-def _stream_ptr(stream):
+def _stream_ptr(stream, device=None):
+    """The cudaStream_t to launch on: ``stream`` (a torch.cuda.Stream or a raw handle), else the current
+    stream of ``device``.  A torch stream that belongs to another device than the tensors is refused."""
     import torch
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
+    sdev = getattr(stream, "device", None)
+    if device is not None and sdev is not None and torch.device(sdev) != torch.device(device):
+        raise ValueError(f"stream is on {sdev}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _on_device(device):
+    """Context that makes ``device`` current for one C-ABI call.  The library resolves the SM count,
+    the shared-memory opt-in and its per-device scratch from the current device, and the default
+    stream is the current device's, so the tensors' device must be current while it runs."""
+    import torch
+    return torch.cuda.device(device)
 
 
 def _ptr(t):
@@ -152,8 +167,9 @@ def fa_fwd(q, k, v, o, lse, causal: bool, scale=None, stream=None) -> None:
     _need(v, "v", torch.bfloat16, dev, (B, H, Nk, d))
     _need(o, "o", torch.bfloat16, dev, (B, H, Nq, d))
     _need(lse, "lse", torch.float32, dev, (B, H, Nq))
-    _check(lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
-                        _scale(scale, d), int(bool(causal)), _stream_ptr(stream)), "fa_fwd")
+    with _on_device(dev):
+        _check(lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                            _scale(scale, d), int(bool(causal)), _stream_ptr(stream, dev)), "fa_fwd")
 
 
 def fa_bwd_workspace_size(B: int, H: int, Nq: int, d: int) -> int:
@@ -175,9 +191,10 @@ def fa_bwd(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal: bool, scale=None,
     _need(lse, "lse", torch.float32, dev, (B, H, Nq))
     _need(workspace, "workspace", torch.uint8, dev)
     fn, name = (lib().fa_bwd_deterministic, "fa_bwd_deterministic") if deterministic else (lib().fa_bwd, "fa_bwd")
-    _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
-              _ptr(workspace), workspace.numel(), B, H, Nq, Nk, d, _scale(scale, d),
-              int(bool(causal)), _stream_ptr(stream)), name)
+    with _on_device(dev):
+        _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+                  _ptr(workspace), workspace.numel(), B, H, Nq, Nk, d, _scale(scale, d),
+                  int(bool(causal)), _stream_ptr(stream, dev)), name)
 
 
 def fa_bwd_deterministic(q, k, v, o, dO, lse, dq, dk, dv, workspace, causal: bool, scale=None, stream=None) -> None:
@@ -206,9 +223,10 @@ def fa_decode_splitkv(q, k_cache, v_cache, seqlens, o, lse, workspace, scale=Non
     if lse is not None:
         _need(lse, "lse", torch.float32, dev, (B, H))
     _need(workspace, "workspace", torch.uint8, dev)
-    _check(lib().fa_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(o), _ptr(lse),
-                                   B, H, d, _scale(scale, d), int(num_splits), _ptr(workspace), workspace.numel(),
-                                   _stream_ptr(stream)), "fa_decode_splitkv")
+    with _on_device(dev):
+        _check(lib().fa_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(o), _ptr(lse),
+                                       B, H, d, _scale(scale, d), int(num_splits), _ptr(workspace), workspace.numel(),
+                                       _stream_ptr(stream, dev)), "fa_decode_splitkv")
 
 
 def fa_decode_splitkv_noalloc(q, k_cache, v_cache, seqlens, o, lse, scale=None, num_splits: int = 0,
@@ -231,9 +249,10 @@ def fa_decode_splitkv_noalloc(q, k_cache, v_cache, seqlens, o, lse, scale=None, 
     _need(o, "o", torch.bfloat16, dev, (B, H, 1, d))
     if lse is not None:
         _need(lse, "lse", torch.float32, dev, (B, H))
-    _check(lib().fa_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(o),
-                                           _ptr(lse), B, H, d, _scale(scale, d), int(num_splits),
-                                           _stream_ptr(stream)), "fa_decode_splitkv_noalloc")
+    with _on_device(dev):
+        _check(lib().fa_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(o),
+                                               _ptr(lse), B, H, d, _scale(scale, d), int(num_splits),
+                                               _stream_ptr(stream, dev)), "fa_decode_splitkv_noalloc")
 
 
 def fa_decode_num_splits(Lmax: int, num_splits: int = 0) -> int:
@@ -257,9 +276,10 @@ def fa_decode_partials(q, k_cache, v_cache, seqlens, part_o, part_ml, scale=None
     _need(seqlens, "seqlens", torch.int32, dev, (B,))
     _need(part_o, "part_o", torch.float32, dev, (B, H, S, d))
     _need(part_ml, "part_ml", torch.float32, dev, (B, H, S, 2))
-    _check(lib().fa_decode_partials(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(part_o),
-                                    _ptr(part_ml), B, H, d, _scale(scale, d), int(num_splits), _stream_ptr(stream)),
-           "fa_decode_partials")
+    with _on_device(dev):
+        _check(lib().fa_decode_partials(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), Lmax, _ptr(part_o),
+                                        _ptr(part_ml), B, H, d, _scale(scale, d), int(num_splits), _stream_ptr(stream, dev)),
+               "fa_decode_partials")
 
 
 def fa_decode_merge(part_o, part_ml, o, lse=None, stream=None) -> None:
@@ -273,8 +293,9 @@ def fa_decode_merge(part_o, part_ml, o, lse=None, stream=None) -> None:
     _need(o, "o", torch.bfloat16, dev, (B, H, 1, d))
     if lse is not None:
         _need(lse, "lse", torch.float32, dev, (B, H))
-    _check(lib().fa_decode_merge(_ptr(part_o), _ptr(part_ml), R, S, _ptr(o), _ptr(lse), B, H, d,
-                                 _stream_ptr(stream)), "fa_decode_merge")
+    with _on_device(dev):
+        _check(lib().fa_decode_merge(_ptr(part_o), _ptr(part_ml), R, S, _ptr(o), _ptr(lse), B, H, d,
+                                     _stream_ptr(stream, dev)), "fa_decode_merge")
 
 
 def _bias_dims(bias, B, H, Nq, Nk, device):
@@ -304,9 +325,10 @@ def fa_fwd_ext(q, k, v, o, lse, bias=None, causal: bool = False, scale=None, dro
     _need(o, "o", torch.bfloat16, dev, (B, H, Nq, d))
     _need(lse, "lse", torch.float32, dev, (B, H, Nq))
     bB, bH = _bias_dims(bias, B, H, Nq, Nk, dev)
-    _check(lib().fa_fwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), bB, bH, _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
-                            _scale(scale, d), int(bool(causal)), float(dropout_p), int(seed) & (2 ** 64 - 1),
-                            int(offset) & 0xFFFFFFFF, _stream_ptr(stream)), "fa_fwd_ext")
+    with _on_device(dev):
+        _check(lib().fa_fwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), bB, bH, _ptr(o), _ptr(lse), B, H, Nq, Nk, d,
+                                _scale(scale, d), int(bool(causal)), float(dropout_p), int(seed) & (2 ** 64 - 1),
+                                int(offset) & 0xFFFFFFFF, _stream_ptr(stream, dev)), "fa_fwd_ext")
 
 
 def fa_bwd_ext(q, k, v, o, dO, lse, dq, dk, dv, workspace, bias=None, causal: bool = False, scale=None,
@@ -323,10 +345,11 @@ def fa_bwd_ext(q, k, v, o, dO, lse, dq, dk, dv, workspace, bias=None, causal: bo
     _need(lse, "lse", torch.float32, dev, (B, H, Nq))
     _need(workspace, "workspace", torch.uint8, dev)
     bB, bH = _bias_dims(bias, B, H, Nq, Nk, dev)
-    _check(lib().fa_bwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(bias), bB, bH, _ptr(dq),
-                            _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), B, H, Nq, Nk, d, _scale(scale, d),
-                            int(bool(causal)), float(dropout_p), int(seed) & (2 ** 64 - 1), int(offset) & 0xFFFFFFFF,
-                            _stream_ptr(stream)), "fa_bwd_ext")
+    with _on_device(dev):
+        _check(lib().fa_bwd_ext(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(bias), bB, bH, _ptr(dq),
+                                _ptr(dk), _ptr(dv), _ptr(workspace), workspace.numel(), B, H, Nq, Nk, d, _scale(scale, d),
+                                int(bool(causal)), float(dropout_p), int(seed) & (2 ** 64 - 1), int(offset) & 0xFFFFFFFF,
+                                _stream_ptr(stream, dev)), "fa_bwd_ext")
 
 
 def _need_e4m3(t, name, device, shape=None):
@@ -347,8 +370,9 @@ def fa_quantize_fp8(x, signs, x8, descale, hadamard: bool = True, stream=None) -
         _need(signs, "signs", torch.float32, dev, (d,))
     _need_e4m3(x8, "x8", dev, (B, H, N, d))
     _need(descale, "descale", torch.float32, dev, (B, H))
-    _check(lib().fa_quantize_fp8(_ptr(x), _ptr(signs), _ptr(x8), _ptr(descale), B, H, N, d, int(bool(hadamard)),
-                                 _stream_ptr(stream)), "fa_quantize_fp8")
+    with _on_device(dev):
+        _check(lib().fa_quantize_fp8(_ptr(x), _ptr(signs), _ptr(x8), _ptr(descale), B, H, N, d, int(bool(hadamard)),
+                                     _stream_ptr(stream, dev)), "fa_quantize_fp8")
 
 
 def fa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, causal: bool, scale=None, stream=None) -> None:
@@ -365,13 +389,25 @@ def fa_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, o, lse, causal: bool
         _need(t, n, torch.float32, dev, (B, H))
     _need(o, "o", torch.bfloat16, dev, (B, H, Nq, d))
     _need(lse, "lse", torch.float32, dev, (B, H, Nq))
-    _check(lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v),
-                            _ptr(o), _ptr(lse), B, H, Nq, Nk, d, _scale(scale, d), int(bool(causal)),
-                            _stream_ptr(stream)), "fa_fwd_fp8")
+    with _on_device(dev):
+        _check(lib().fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v),
+                                _ptr(o), _ptr(lse), B, H, Nq, Nk, d, _scale(scale, d), int(bool(causal)),
+                                _stream_ptr(stream, dev)), "fa_fwd_fp8")
 
 
-def fa_get_device_error(stream=None) -> int:
-    return int(lib().fa_get_device_error(_stream_ptr(stream)))
+def fa_debug_set_wait_limit(limit_ns: int, device=None) -> None:
+    """Test hook (see include/fa.h: fa_debug_set_wait_limit): the limit of every pipeline wait on
+    ``device`` (default: current), 0 restoring the default 2 s."""
+    with _on_device(device):
+        _check(lib().fa_debug_set_wait_limit(int(limit_ns)), "fa_debug_set_wait_limit")
+
+
+def fa_get_device_error(stream=None, device=None) -> int:
+    """Synchronise the stream and read and clear the device status word (see include/fa.h: fa_get_device_error)
+    of ``device`` (default: the stream's device, else the current device)."""
+    dev = device if device is not None else getattr(stream, "device", None)
+    with _on_device(dev):
+        return int(lib().fa_get_device_error(_stream_ptr(stream, dev)))
 
 
 # ------------------------------------------------------------------------------ conveniences

@@ -10,7 +10,7 @@
 // "Parallel random numbers: as easy as 1, 2, 3", SC 2011) keyed by the 64-bit seed.  One call
 // covers 4 queries x 4 keys of one (batch, head): counter = (key / 4, query / 4, b * H + h,
 // offset); byte (key % 4) of word (query % 4) is the entry's random byte u, and the entry is
-// kept iff u >= p8 (p8 = round(256 p)).  Kept weights are scaled by 256 / (256 - p8).
+// kept iff u >= p8 (p8 = floor(256 p + 1/2)).  Kept weights are scaled by 256 / (256 - p8).
 //
 // Lane layout: in the forward a thread owns a query row (4 consecutive lanes = one query quad);
 // in the backward a thread owns a key row (4 consecutive lanes = one key quad).  Each lane of a

@@ -144,7 +144,8 @@ void set_ext(P& p, const ExtArgs* ext) {
 fa_status make_ext(ExtArgs* ext, const void* bias, int bias_B, int bias_H, int B, int H, int Nq, int Nk,
                    float dropout_p, unsigned long long seed, unsigned int offset) {
   if (!(dropout_p >= 0.f && dropout_p < 1.f)) return FA_ERR_INVALID_ARG;
-  long r = std::lround(256.0 * (double)dropout_p);
+  // p8 = floor(256 p + 1/2): a tie (256 p exactly half-way between two integers) goes up.
+  const long r = (long)std::floor(256.0 * (double)dropout_p + 0.5);
   const uint32_t p8 = (uint32_t)(r > 255 ? 255 : r);
   ext->drop = fa::DropoutCfg{p8, (float)(256.0 / (256.0 - (double)p8)), (uint32_t)(seed & 0xffffffffull),
                              (uint32_t)(seed >> 32), offset};
@@ -443,6 +444,13 @@ static fa_status bwd_entry(const void* q, const void* k, const void* v, const vo
   if (need > 0 && (!workspace || ws_bytes < need)) return FA_ERR_WORKSPACE;
   if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FA_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!has_q) {
+    // No query row: no score touches any key, so dK = dV = 0 (nothing else is read or written).
+    const size_t bytes = (size_t)BH * Nk * d * sizeof(__nv_bfloat16);
+    if (cudaMemsetAsync(dk, 0, bytes, s) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, s) != cudaSuccess)
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
   return d == 64 ? launch_bwd<64>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s, deterministic,
                                   ext)
                  : launch_bwd<128>(q, k, v, o, dO, lse, dq, dk, dv, workspace, (int)BH, Nq, Nk, scale, causal, s,
@@ -589,6 +597,14 @@ fa_status fa_get_device_error(void* stream) {
     if (cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
   }
   return v == 0 ? FA_OK : static_cast<fa_status>(v);
+}
+
+fa_status fa_debug_set_wait_limit(unsigned long long limit_ns) {
+  const unsigned long long lim = limit_ns == 0 ? fa::kWaitLimitNs : limit_ns;
+  const uint32_t hint = (uint32_t)(lim < fa::kSuspendHintNs ? lim : fa::kSuspendHintNs);
+  if (cudaMemcpyToSymbol(fa::c_wait_limit_ns, &lim, sizeof(lim)) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(fa::c_suspend_hint_ns, &hint, sizeof(hint)) != cudaSuccess) return FA_ERR_CUDA;
+  return FA_OK;
 }
 
 const char* fa_status_string(fa_status status) {

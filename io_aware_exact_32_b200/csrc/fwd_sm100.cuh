@@ -34,13 +34,6 @@ namespace fa {
 
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// One in kPolyEvery pairs of exponentials is evaluated on the FMA pipe instead of MUFU
-// (0 = all on MUFU).  Off by default: measured on B200, moving a third or a quarter of the
-// exponentials off MUFU did not shorten the forward at d = 128.
-#ifndef FA_FWD_POLY_EVERY
-#define FA_FWD_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = FA_FWD_POLY_EVERY;
 
 template <int D, bool F8 = false>
 struct FwdTraits {
@@ -208,6 +201,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
   const bool two = p.tiles == 2;
   const int q0 = unit * 128 * p.tiles;
   const int n_kv = fwd_num_kv_tiles(q0, 128 * p.tiles, p.Nq, p.Nk, p.causal);
+  int issued = 0;  // K/V loads started by the TMA producer (its lane 0), for the teardown
 
   if (threadIdx.x == 0) {
     mbar_init(bar(T::BAR_Q), 1);
@@ -343,12 +337,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const float2 x = ffma2(make_float2(src[2 * c], src[2 * c + 1]), sc2, nb2);
-            float2 e;
-            if (kPolyEvery > 0 && (c % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1) {
-              e = exp2_poly2(x);
-            } else {
-              e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            }
+            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
             pk[c] = pack_bf16x2(e.x, e.y);
             sum_e[c & 1] = fadd2(sum_e[c & 1], e);
             sum_r[c & 1] = fadd2(sum_r[c & 1], make_float2(bf16lo_to_f32(pk[c]), bf16hi_to_f32(pk[c])));
@@ -540,13 +529,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
         fwd_issue_pv<D, F8>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, n_kv - 1 > 0);
         mma_commit_w(bar(T::BAR_O_DONE + 1));
       }
-      if (!ok) {
-        *abort_flag = 1;
-        // Let every MMA already issued finish before the CTA releases its tensor memory.
-        mma_commit_w(bar(T::BAR_DRAIN));
-        const volatile int never = 0;
-        warp_wait(bar(T::BAR_DRAIN), 0, &never);
-      }
+      if (!ok) *abort_flag = 1;
     }
     __syncwarp();
   } else {
@@ -559,7 +542,6 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
                       q0 + 128 * t, bh);
       const int total_loads = 2 * n_kv;
       bool ok = true;
-      int issued = 0;
       for (int idx = 0; idx < total_loads; ++idx) {
         const int s = idx % T::NS;
         if (!(ok = mbar_wait(bar(T::BAR_KV_EMPTY + s), ((idx / T::NS) & 1) ^ 1, abort_flag))) break;
@@ -570,24 +552,30 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
                       T::BOX_COLS * b, 128 * (idx >> 1), bh);
         issued = idx + 1;
       }
-      if (!ok) {
-        *abort_flag = 1;
-        // Wait (bounded) for the copies still in flight before shared memory is given back.
-        const volatile int never = 0;
-        for (int idx = max(0, issued - T::NS); idx < issued; ++idx)
-          mbar_wait(bar(T::BAR_KV_FULL + idx % T::NS), (idx / T::NS) & 1, &never);
-        mbar_wait(bar(T::BAR_Q), 0, &never);
-      }
+      if (!ok) *abort_flag = 1;
     }
     __syncwarp();
   }
 
-teardown:
+  // Teardown.  On the normal path every copy and MMA has been consumed by now.  If any warp gave
+  // up, the others have stopped too (they poll the abort flag); then the CTA still waits for its
+  // own work in flight (fixed-limit waits): the MMAs before tensor memory is freed, the copies
+  // before shared memory is given back with the CTA's exit.
+  if (warp < 8) tmem_st_wait();
   tc_fence_before();
   __syncthreads();
+  const bool aborted = *abort_flag != 0;
   if (warp == 8) {
+    if (aborted) {
+      mma_commit_w(bar(T::BAR_DRAIN));
+      warp_drain_wait(bar(T::BAR_DRAIN), 0);
+    }
     tc_fence_after();
     tmem_dealloc(tmem_base, T::TMEM_COLS);
+  } else if (warp == 9 && lane == 0 && aborted) {
+    for (int idx = max(0, issued - T::NS); idx < issued; ++idx)
+      drain_wait(bar(T::BAR_KV_FULL + idx % T::NS), (idx / T::NS) & 1);
+    drain_wait(bar(T::BAR_Q), 0);
   }
 }
 

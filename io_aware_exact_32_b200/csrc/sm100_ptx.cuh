@@ -62,27 +62,50 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 // the warps that share their scheduler.
 constexpr uint32_t kSuspendHintNs = 500000;
 
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// Limit and suspend hint of the pipeline waits.  They stay at kWaitLimitNs / kSuspendHintNs; only
+// the test hook fa_debug_set_wait_limit lowers them, so that a test can make a healthy kernel's
+// waits run out and exercise the give-up path.  Teardown waits (drain_wait) always use the fixed
+// constants: a CTA that gave up still waits for its own copies and MMAs before it frees anything.
+__constant__ unsigned long long c_wait_limit_ns = kWaitLimitNs;
+__constant__ uint32_t c_suspend_hint_ns = kSuspendHintNs;
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
 
 // Waits for completion of the phase with the given parity.  Gives up (returns
-// false) after kWaitLimitNs, or once *abort is set by another warp (checked each
+// false) after the wait limit, or once *abort is set by another warp (checked each
 // time a suspended try_wait returns without completion).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = c_suspend_hint_ns;
+  if (mbar_try_wait(bar, parity, hint)) return true;
+  const unsigned long long t0 = global_timer_ns();
+  const unsigned long long limit = c_wait_limit_ns;
+  while (true) {
+    if (mbar_try_wait(bar, parity, hint)) return true;
+    if (*abort) return false;
+    if (global_timer_ns() - t0 > limit) {
+      record_timeout();
+      return false;
+    }
+  }
+}
+
+// Teardown wait: for this CTA's own copies or MMAs in flight, with the fixed limit and no abort
+// flag.  Returns false (and records a timeout) only if they never complete.
+__device__ __forceinline__ bool drain_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity, kSuspendHintNs)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
+    if (mbar_try_wait(bar, parity, kSuspendHintNs)) return true;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       record_timeout();
       return false;
@@ -236,6 +259,9 @@ __device__ __forceinline__ void mma_commit_w(uint32_t bar) {
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const volatile int* abort) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
+__device__ __forceinline__ bool warp_drain_wait(uint32_t bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, drain_wait(bar, parity));
+}
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -323,31 +349,6 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
-}
-
-// 2^x on the FMA pipe for a pair of values (frees the MUFU unit, which the exponentials of the
-// softmax otherwise saturate).  Cody-Waite style range reduction: x = n + f with n = round(x)
-// obtained by adding 1.5 * 2^23 (which leaves round(x) in the low mantissa bits) and
-// f in [-0.5, 0.5]; 2^f from a cubic fitted to 2^f on [-0.5, 0.5] by iteratively reweighted
-// least squares on the relative error (our own fit; max relative error 7.5e-5 in fp32 Horner
-// form, far below the 2^-9 of the bf16 rounding that follows); 2^n is added to the exponent
-// field.  Inputs below -125 (including -inf) return exactly 0: they are clamped first so the
-// exponent field cannot wrap, then zeroed.  Valid for x <= 127.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.99992812f, c1 = 0.69326097f, c2 = 0.24261054f, c3 = 0.05517132f;
-  const bool zx = x.x < -125.f, zy = x.y < -125.f;
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = fadd2(x, make_float2(kRound, kRound));
-  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
-  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
-  float2 p = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
-  p = ffma2(p, f, make_float2(c1, c1));
-  p = ffma2(p, f, make_float2(c0, c0));
-  const uint32_t bx = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
-  const uint32_t by = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
-  return make_float2(zx ? 0.f : __uint_as_float(bx), zy ? 0.f : __uint_as_float(by));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

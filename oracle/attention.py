@@ -52,6 +52,8 @@ __all__ = [
     "attention_backward",
     "attention_backward_q_rows",
     "attention_backward_kv_rows",
+    "attention_row_block",
+    "attention_backward_full_head",
     "decode_forward",
 ]
 
@@ -267,6 +269,71 @@ def attention_backward_kv_rows(q_head, k_head, v_head, do_head, keys, scale: flo
         dv += p_sel.T @ doh[r]
         dk += scale * (ds_sel.T @ qh[r])
     return dk, dv
+
+
+def attention_row_block(q_head, k_head, v_head, do_head, r0: int, r1: int, scale: float, causal: bool):
+    """Forward and backward of the query rows [r0, r1) of one head, each row with its whole score row.
+
+    Returns (O, LSE, dQ) of those rows and their terms of dK and dV: dK = scale * sum_i dS_i^T q_i and
+    dV = sum_i P_i^T dO_i are sums over query rows, so the terms of all row blocks add up to the full
+    dK and dV (the plain definition, split along the sum).  Under the causal mask the keys past the
+    block's last visible key have P = 0 and contribute nothing, so they are left out of the products
+    and the dK, dV terms are returned for keys [0, kend) only (kend = the number of keys the block
+    can see; Nk without the mask).
+    """
+    nq, nk = q_head.shape[0], k_head.shape[0]
+    kend = nk if not causal else max(0, min(nk, (r1 - 1) + (nk - nq) + 1))
+    q = np.asarray(q_head[r0:r1], np.float64)
+    k = np.asarray(k_head[:kend], np.float64)
+    v = np.asarray(v_head[:kend], np.float64)
+    do = np.asarray(do_head[r0:r1], np.float64)
+    if kend == 0:
+        return (np.zeros((r1 - r0, v_head.shape[1])), np.full(r1 - r0, -np.inf), np.zeros_like(q),
+                np.zeros((0, k_head.shape[1])), np.zeros((0, v_head.shape[1])))
+    s = scale * (q @ k.T)
+    if causal:
+        s = np.where(causal_visible(nq, nk, rows=np.arange(r0, r1), cols=np.arange(kend)), s, -np.inf)
+    p, lse = softmax_rows(s)
+    o = p @ v
+    dp = do @ v.T
+    drow = np.sum(do * o, axis=-1)
+    ds = p * (dp - drow[:, None])
+    dq = scale * (ds @ k)
+    return o, lse, dq, scale * (ds.T @ q), p.T @ do
+
+
+def attention_backward_full_head(q_head, k_head, v_head, do_head, scale: float, causal: bool,
+                                 block: int = 256, workers: int = 1):
+    """dQ, dK, dV (and O, LSE) of one whole head, for sizes whose N x N matrices do not fit in host
+    memory: the row blocks of ``attention_row_block`` summed.  ``workers`` > 1 evaluates the blocks
+    on that many threads (numpy releases the interpreter lock in its kernels); the sums are the same
+    up to the order of float64 additions."""
+    import threading
+    nq, nk = q_head.shape[0], k_head.shape[0]
+    o = np.zeros((nq, v_head.shape[1]))
+    lse = np.zeros(nq)
+    dq = np.zeros((nq, q_head.shape[1]))
+    dk = np.zeros((nk, k_head.shape[1]))
+    dv = np.zeros((nk, v_head.shape[1]))
+    lock = threading.Lock()
+
+    def one(r0):
+        r1 = min(nq, r0 + block)
+        o[r0:r1], lse[r0:r1], dq[r0:r1], dk_t, dv_t = attention_row_block(q_head, k_head, v_head, do_head, r0, r1,
+                                                                          scale, causal)
+        with lock:
+            dk[:len(dk_t)] += dk_t
+            dv[:len(dv_t)] += dv_t
+
+    starts = range(0, nq, block)
+    if workers > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(workers) as ex:
+            list(ex.map(one, starts))
+    else:
+        for r0 in starts:
+            one(r0)
+    return o, lse, dq, dk, dv
 
 
 def decode_forward(q, k_cache, v_cache, seqlens, scale: float):

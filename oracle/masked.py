@@ -28,11 +28,15 @@ Readings where the pages are silent:
   One call covers a block of 4 queries x 4 keys of one (batch, head):
   counter = (key // 4, query // 4, b * H + h, offset), key = (seed mod 2^32,
   seed // 2^32); output word (query mod 4), byte (key mod 4) (least significant
-  first) is that entry's random byte u.  p is used as p8 = round(256 p) in
-  [0, 255]: the entry is kept iff u >= p8, and the kept weights are scaled by
+  first) is that entry's random byte u.  p is used as the byte threshold
+  p8 = floor(256 p + 1/2) in [0, 255], with p the float32 value the C ABI
+  receives (a tie, 256 p exactly half-way between two integers, goes up): the
+  entry is kept iff u >= p8, and the kept weights are scaled by
   256 / (256 - p8).
 """
 from __future__ import annotations
+
+import math
 
 import numpy as np
 
@@ -73,10 +77,11 @@ def philox(counter, key, rounds: int = 10, params=PHILOX4x32):
 
 
 def dropout_p8(p: float) -> int:
-    """The byte threshold for dropout probability p in [0, 1)."""
+    """The byte threshold floor(256 p + 1/2) for dropout probability p in [0, 1), p taken as float32."""
     if not (0.0 <= p < 1.0):
         raise ValueError("dropout probability must be in [0, 1)")
-    return min(255, int(round(256.0 * p)))
+    p32 = float(np.float32(p))
+    return min(255, int(math.floor(256.0 * p32 + 0.5)))
 
 
 def dropout_keep(B: int, H: int, Nq: int, Nk: int, p8: int, seed: int, offset: int = 0,

@@ -1,6 +1,7 @@
 """The C-ABI library: it loads, exports every call include/fa.h declares, and
 rejects bad arguments on the host before touching the GPU (no compute calls)."""
 import ctypes
+import math
 import os
 import re
 
@@ -215,3 +216,93 @@ def test_product_package_never_imports_the_oracle():
                 src = open(os.path.join(root, f), encoding="utf-8").read()
                 assert not re.search(r"^\s*(from|import)\s+oracle\b", src, flags=re.M), f
                 assert "oracle/" not in src, f
+
+
+class _FakeTensor:
+    """Shape, device and pointer of a tensor, without memory (never dereferenced: the library is faked)."""
+
+    def __init__(self, shape, device):
+        self.shape = tuple(shape)
+        self.device = device
+
+    def data_ptr(self):
+        return 0x10000
+
+    def numel(self):
+        return math.prod(self.shape)
+
+
+def test_binding_makes_the_tensors_device_current(monkeypatch):
+    """Each C-ABI call runs with the tensors' device current (the library resolves the SM count, its
+    shared-memory opt-in, its scratch and the default stream from the current device)."""
+    torch = pytest.importorskip("torch")
+    current = ["cuda:0"]
+    calls = []
+
+    class Guard:
+        def __init__(self, dev):
+            self.dev = dev
+
+        def __enter__(self):
+            self.prev = current[0]
+            current[0] = str(self.dev)
+
+        def __exit__(self, *exc):
+            current[0] = self.prev
+
+    class FakeLib:
+        def __getattr__(self, name):
+            def call(*args):
+                calls.append((name, current[0]))
+                return 0
+            return call
+
+    monkeypatch.setattr(fa, "_on_device", Guard)
+    monkeypatch.setattr(fa, "lib", lambda: FakeLib())
+    monkeypatch.setattr(fa, "_need", lambda *a, **k: None)
+    monkeypatch.setattr(fa, "_stream_ptr", lambda s, d=None: ctypes.c_void_p(0))
+    dev = torch.device("cuda", 1)
+    t = _FakeTensor((1, 2, 128, 64), dev)
+    lse = _FakeTensor((1, 2, 128), dev)
+    fa.fa_fwd(t, t, t, t, lse, causal=True)
+    fa.fa_bwd(t, t, t, t, t, lse, t, t, t, _FakeTensor((1 << 20,), dev), causal=True)
+    fa.fa_fwd_ext(t, t, t, t, lse, None, True)
+    one = _FakeTensor((1, 2, 1, 64), dev)
+    fa.fa_decode_splitkv(one, t, t, _FakeTensor((1,), dev), one, None, _FakeTensor((1 << 20,), dev))
+    assert [n for n, _ in calls] == ["fa_fwd", "fa_bwd", "fa_fwd_ext", "fa_decode_splitkv"]
+    assert all(d == "cuda:1" for _, d in calls), calls
+    assert current[0] == "cuda:0"
+
+
+def test_binding_refuses_a_stream_of_another_device():
+    torch = pytest.importorskip("torch")
+
+    class Stream:
+        device = torch.device("cuda", 1)
+        cuda_stream = 0
+
+    with pytest.raises(ValueError, match="stream"):
+        fa._stream_ptr(Stream(), torch.device("cuda", 0))
+    assert fa._stream_ptr(Stream(), torch.device("cuda", 1)).value in (None, 0)
+
+
+def test_bwd_without_query_rows_needs_only_dk_dv(L):
+    """Nq == 0, Nk > 0: the only outputs are dK = dV = 0, so q, o, dO, lse, dq and the workspace may be
+    NULL.  Validation accepts the call; with no GPU in this process the zeroing memset itself fails
+    (FA_ERR_CUDA).  Skipped where a GPU exists: the fake pointers would reach a device memset there
+    (the GPU half is tests/test_parity_bwd.py::test_no_query_rows_gives_zero_dk_dv)."""
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("fake pointers must not reach a device")
+    st = L.fa_bwd(NULL, A16, A16, NULL, NULL, NULL, NULL, A16, A16, NULL, 0, 1, 2, 0, 128, 64, 0.125, 1, NULL)
+    assert st == 5, fa.fa_status_string(st)
+    assert L.fa_bwd(NULL, NULL, A16, NULL, NULL, NULL, NULL, A16, A16, NULL, 0, 1, 2, 0, 128, 64, 0.125, 1,
+                    NULL) == 1   # k is still needed
+
+
+def test_wait_limit_hook_without_a_device(L):
+    """The test hook copies to device constant memory; with no GPU that copy fails cleanly."""
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("changes the device's wait limit; covered by tests/test_bounded_wait.py")
+    assert L.fa_debug_set_wait_limit(0) == 5

@@ -1,0 +1,57 @@
+"""The give-up path of the kernels' bounded waits, exercised without any fault.
+
+Every wait in the kernels gives up after a time limit (2 s by default): the CTA
+records FA_ERR_TIMEOUT in the device status word, the other warps of the CTA
+see its abort flag and stop, and the teardown still waits (with the fixed 2 s
+limit) for the CTA's own copies and MMAs in flight before it frees its tensor
+memory and exits.  Here the test hook fa_debug_set_wait_limit lowers the
+limit to 300 ns, so the waits of a healthy causal forward run out; the test
+checks that fa_get_device_error reports the timeout, restores the limit, and
+checks that the next forward on the same device matches the float64 oracle
+(nothing was left allocated or half-written that it could trip over).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import io_aware_exact_32_b200 as fa
+from io_aware_exact_32_b200 import workloads as W
+from oracle import attention as A
+import gpu_common as gc
+from tolerances import check_lse, check_o
+
+pytestmark = pytest.mark.gpu
+
+FA_ERR_TIMEOUT = 6
+
+
+def test_waits_give_up_and_the_device_stays_usable():
+    B, H, N, d = 1, 16, 4096, 128
+    x = W.make_attention_inputs(B, H, N, N, d, seed=91, with_do=False)
+    q, k, v = gc.to_dev(x["q"], x["k"], x["v"])
+    scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=gc.DEV)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    fa.fa_debug_set_wait_limit(300)
+    try:
+        fa.fa_fwd(q, k, v, o, lse, True, scale)
+        torch.cuda.synchronize()
+        status = fa.fa_get_device_error()
+    finally:
+        fa.fa_debug_set_wait_limit(0)
+    assert status == FA_ERR_TIMEOUT, status
+
+    o2, lse2 = fa.attention_forward(q, k, v, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    rows = gc.sample_rows(N, 48, 5)
+    for h in (0, H - 1):
+        ro, rl = A.attention_forward_rows(gc.f64(x["q"][0, h]), gc.f64(x["k"][0, h]), gc.f64(x["v"][0, h]),
+                                          rows, scale, True)
+        check_o(gc.f64(o2[0, h, rows]), ro, f"O[{h}]")
+        check_lse(gc.f64(lse2[0, h, rows]), rl, f"LSE[{h}]")
+    assert np.isfinite(gc.f64(o2)).all()

@@ -417,3 +417,69 @@ def test_correct_mutant_template_passes():
     """The mutant templates with no planted mistake pass every pin (the pins are not vacuous)."""
     assert all(pin(_fwd_mutant("none")) for pin in FORWARD_PINS)
     assert all(pin(_bwd_mutant("none")) for pin in BACKWARD_PINS)
+
+
+# ----------------------------------------------------------------------------------------
+# the whole-head backward by row blocks (used for full-size gradient parity) is pinned by the
+# same pins as the plain backward: finite differences, torch autograd, the gradient sums and the
+# hand-worked golden, at block sizes that cut the rows (and, under the causal mask, the key
+# range each block keeps) at every position
+# ----------------------------------------------------------------------------------------
+def _full_head_bwd(block, workers):
+    def bwd(q, k, v, do, scale, causal):
+        return A.attention_backward_full_head(q, k, v, do, scale, causal, block=block, workers=workers)[2:]
+    return bwd
+
+
+def _full_head_fwd(block):
+    def fwd(q, k, v, scale, causal):
+        do = np.zeros((q.shape[0], v.shape[1]))
+        return A.attention_backward_full_head(q, k, v, do, scale, causal, block=block)[:2]
+    return fwd
+
+
+@pytest.mark.parametrize("block,workers", [(1, 1), (2, 1), (3, 2), (64, 1)])
+@pytest.mark.parametrize("pin", BACKWARD_PINS, ids=lambda f: f.__name__)
+def test_full_head_backward_pin(pin, block, workers):
+    assert pin(_full_head_bwd(block, workers))
+
+
+@pytest.mark.parametrize("block", [1, 2, 5])
+@pytest.mark.parametrize("pin", FORWARD_PINS, ids=lambda f: f.__name__)
+def test_full_head_forward_pin(pin, block):
+    assert pin(_full_head_fwd(block))
+
+
+def test_full_head_rows_with_no_key():
+    """Causal, Nq > Nk: blocks whose rows see no key give O = 0, LSE = -inf, dQ = 0."""
+    nq, nk, d = 9, 4, 3
+    q, k, v, do = _rand((nq, d), 130), _rand((nk, d), 131), _rand((nk, d), 132), _rand((nq, d), 133)
+    o, lse, dq, dk, dv = A.attention_backward_full_head(q, k, v, do, 0.5, True, block=2)
+    ro, rl = A.attention_forward_head(q, k, v, 0.5, True)
+    rq, rk, rv = A.attention_backward_head(q, k, v, do, 0.5, True)
+    assert np.all(o[:5] == 0) and np.all(np.isneginf(lse[:5])) and np.all(dq[:5] == 0)
+    assert np.allclose(o, ro, atol=1e-14) and np.array_equal(np.isneginf(lse), np.isneginf(rl))
+    assert np.allclose(dq, rq, atol=1e-13) and np.allclose(dk, rk, atol=1e-13) and np.allclose(dv, rv, atol=1e-13)
+
+
+def test_full_head_mutant_dropping_the_last_visible_key_is_caught():
+    """A plausible slip in the causal key range of a row block (one key short) fails the autograd pin."""
+    real = A.attention_row_block
+
+    def short(q_head, k_head, v_head, do_head, r0, r1, scale, causal):
+        nq, nk = q_head.shape[0], k_head.shape[0]
+        kend = nk if not causal else max(0, min(nk, (r1 - 1) + (nk - nq)))   # one key short
+        q, k, v, do = q_head[r0:r1], k_head[:kend], v_head[:kend], do_head[r0:r1]
+        s = scale * (q @ k.T)
+        if causal:
+            s = np.where(A.causal_visible(nq, nk, rows=np.arange(r0, r1), cols=np.arange(kend)), s, -np.inf)
+        p, lse = A.softmax_rows(s)
+        o = p @ v
+        ds = p * (do @ v.T - np.sum(do * o, axis=-1)[:, None])
+        return o, lse, scale * (ds @ k), scale * (ds.T @ q), p.T @ do
+
+    A.attention_row_block = short
+    try:
+        assert not pin_torch_autograd(_full_head_bwd(2, 1))
+    finally:
+        A.attention_row_block = real

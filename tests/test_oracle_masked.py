@@ -297,3 +297,15 @@ def _bwd_dp_without_dropout(q, k, v, do, bias, scale, causal, keep=None, p8=0):
 def test_pins_reject_planted_mistakes(pin, impl):
     with pytest.raises(AssertionError):
         pin(impl)
+
+
+def test_dropout_threshold_rounding():
+    """p8 = floor(256 p + 1/2) of the float32 p: worked by hand, ties included.  A tie is a p whose
+    256 p is an odd multiple of 1/2 and exact in float32 (p = 2.5 / 256 gives 3, not Python's
+    round-half-even 2)."""
+    cases = {0.0: 0, 0.1: 26, 0.5: 128, 0.9: 230, 2.5 / 256: 3, 3.5 / 256: 4, 0.5 / 256: 1,
+             254.5 / 256: 255, 255.4 / 256: 255, 0.99: 253}
+    for p, want in cases.items():
+        assert M.dropout_p8(p) == want, (p, M.dropout_p8(p), want)
+    with pytest.raises(ValueError):
+        M.dropout_p8(1.0)

@@ -15,6 +15,7 @@ import torch
 
 import io_aware_exact_32_b200 as fa
 from io_aware_exact_32_b200 import workloads as W
+from oracle import attention as A
 from oracle import masked as M
 import gpu_common as gc
 from tolerances import check_grad, check_lse, check_o
@@ -83,7 +84,7 @@ def test_ext_matches_oracle(B, H, Nq, Nk, d, causal, bdims, p):
     check_grad(gc.f64(dv), rv, "dV")
 
 
-@pytest.mark.parametrize("p", [0.1, 0.5, 0.9])
+@pytest.mark.parametrize("p", [0.1, 0.5, 0.9, 2.5 / 256])   # 2.5 / 256: a rounding tie (p8 = 3)
 def test_dropout_pattern_is_the_oracle_one(p):
     """Q = 0 (uniform weights, no bias), one-hot rows: the forward's O and the backward's dV show each
     decision of every (batch, head) exactly."""
@@ -100,6 +101,39 @@ def test_dropout_pattern_is_the_oracle_one(p):
     assert np.array_equal(bwd_kept, keep), int((bwd_kept != keep).sum())
     want = 256.0 / (256 - p8) / N
     assert np.allclose(gc.f64(o)[keep], want, rtol=2 ** -8)
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", [
+    (2, 32, 600, 128, True),   # enough CTAs for two 128-row query tiles per CTA; ragged last tile
+    (1, 2, 600, 64, False),    # one query tile per CTA, its key tiles split between the two groups
+    (1, 3, 384, 128, False),
+])
+def test_dropout_pattern_across_tiles(B, H, N, d, causal):
+    """Every decision of an N x N pattern, across query-tile and key-tile boundaries, equals the oracle's.
+
+    Q = 0 makes the weights uniform over the visible keys.  V one-hot on a window of d keys makes the
+    forward's O show the decisions of those keys (O[i, c] != 0 iff key w0 + c is kept and visible),
+    and dO one-hot on a window of d queries makes the backward's dV show the decisions of those
+    queries (dV[j, c] != 0 iff entry (w0 + c, j) is kept and visible); windows cover every key and
+    every query."""
+    p = 0.3
+    p8 = M.dropout_p8(p)
+    keep = M.dropout_keep(B, H, N, N, p8, SEED, OFFSET)
+    vis = A.causal_visible(N, N) if causal else np.ones((N, N), dtype=bool)
+    want = keep & vis[None, None]
+    k = W.make_attention_inputs(B, H, N, N, d, 3, with_do=False)["k"]
+    q = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+    fwd_seen = np.zeros((B, H, N, N), dtype=bool)
+    bwd_seen = np.zeros((B, H, N, N), dtype=bool)
+    for w0 in range(0, N, d):
+        kw = min(d, N - w0)
+        onehot = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+        onehot[:, :, torch.arange(w0, w0 + kw), torch.arange(kw)] = 1.0
+        o, _, (_, _, dv) = run_ext({"q": q, "k": k, "v": onehot, "do": onehot}, None, causal, 0.125, p)
+        fwd_seen[:, :, :, w0:w0 + kw] = gc.f64(o)[..., :kw] != 0
+        bwd_seen[:, :, w0:w0 + kw, :] = (gc.f64(dv)[..., :kw] != 0).transpose(0, 1, 3, 2)
+    assert np.array_equal(fwd_seen, want), int((fwd_seen != want).sum())
+    assert np.array_equal(bwd_seen, want), int((bwd_seen != want).sum())
 
 
 def test_without_bias_or_dropout_matches_the_plain_path():

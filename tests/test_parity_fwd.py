@@ -99,8 +99,10 @@ def _sampled_check(cfg, causal, rows_per_head, seed):
 
 @pytest.mark.parametrize("cfg", W.SWEEP, ids=lambda c: c.name)
 def test_sweep_full_size_sampled(cfg):
-    _sampled_check(cfg, True, rows_per_head=24, seed=7)
+    _sampled_check(cfg, True, rows_per_head=64, seed=7)
 
 
 def test_long_context_sampled():
-    _sampled_check(W.LONG, True, rows_per_head=40, seed=9)
+    """512 sampled rows of every head (rows 0, 1 and N-1 and queries at peaked key positions among
+    them); the whole of heads 0 and 15 is compared in tests/test_parity_bwd.py."""
+    _sampled_check(W.LONG, True, rows_per_head=512, seed=9)
