@@ -114,6 +114,7 @@ struct BwdParams {
   // Bias and dropout instantiation only (as in FwdParams).
   const __nv_bfloat16* bias;
   long long bias_sb, bias_sh;
+  int bias_pb, bias_ph;
   int H;
   DropoutCfg drop;
 };
@@ -190,7 +191,8 @@ template <int D, bool DQ = true, bool EXT = false>
 __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                       const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
+                       const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmB,
+                       const BwdParams p) {
   using T = BwdTraits<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -246,6 +248,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmDO);
     if (T::SEP_DQ) tma_prefetch_desc(&tmDQ);
+    if (EXT && p.bias != nullptr) tma_prefetch_desc(&tmB);
   }
   tc_fence_before();
   __syncthreads();
@@ -667,6 +670,14 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           tma_load_3d(dst + T::TILE_BYTES + b * T::BOX_BYTES, &tmDO, bar(T::BAR_QD_FULL + s), 64 * b, q0, bh);
         }
         issued = it + 1;
+        if constexpr (EXT) {
+          // Warm the L2 with this block's bias tile (the P/dS threads read its key columns with plain
+          // loads once the block's stage is consumed).
+          if (p.bias != nullptr) {
+            const int plane = (bh / p.H) * p.bias_pb + (bh % p.H) * p.bias_ph;
+            for (int b = 0; b < 2; ++b) tma_prefetch_l2_3d(&tmB, k0 + 64 * b, q0, plane);
+          }
+        }
       }
       if (!ok) {
         *abort_flag = 1;

@@ -70,6 +70,21 @@ bool make_map_3d_f32(CUtensorMap* map, void* base, int D, int N, long long BH) {
   return r == CUDA_SUCCESS;
 }
 
+// [planes, Nq, Nk] bf16 bias viewed as {Nk, Nq, planes}; box = 64 keys x 128 query rows x 1, used only
+// for L2 prefetches.  Rows past Nq and keys past Nk are clipped.
+bool make_map_bias(CUtensorMap* map, const void* base, int Nk, int Nq, long long planes) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)Nk, (cuuint64_t)Nq, (cuuint64_t)planes};
+  cuuint64_t strides[2] = {(cuuint64_t)Nk * 2, (cuuint64_t)Nq * Nk * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -127,15 +142,26 @@ int decode_chunk(int Lmax, int S) {
 struct ExtArgs {
   const __nv_bfloat16* bias;  // null: no bias
   long long sb, sh;           // element strides of b and h in the bias (0 where broadcast)
+  int pb, ph;                 // the same strides in [Nq, Nk] planes
+  long long planes;           // bias_B * bias_H
   int H;
   fa::DropoutCfg drop;
 };
+
+// The bias tensor map of an extended call (all zero when there is no bias: never read then).
+bool ext_bias_map(CUtensorMap* map, const ExtArgs* ext, int Nq, int Nk) {
+  std::memset(map, 0, sizeof(*map));
+  if (!ext || !ext->bias) return true;
+  return make_map_bias(map, ext->bias, Nk, Nq, ext->planes);
+}
 
 template <typename P>
 void set_ext(P& p, const ExtArgs* ext) {
   p.bias = ext ? ext->bias : nullptr;
   p.bias_sb = ext ? ext->sb : 0;
   p.bias_sh = ext ? ext->sh : 0;
+  p.bias_pb = ext ? ext->pb : 0;
+  p.bias_ph = ext ? ext->ph : 0;
   p.H = ext ? ext->H : 1;
   p.drop = ext ? ext->drop : fa::DropoutCfg{0u, 1.f, 0u, 0u, 0u};
 }
@@ -152,6 +178,8 @@ fa_status make_ext(ExtArgs* ext, const void* bias, int bias_B, int bias_H, int B
   ext->H = H;
   ext->bias = static_cast<const __nv_bfloat16*>(bias);
   ext->sb = ext->sh = 0;
+  ext->pb = ext->ph = 0;
+  ext->planes = 1;
   if (bias) {
     if ((bias_B != 1 && bias_B != B) || (bias_H != 1 && bias_H != H)) return FA_ERR_INVALID_ARG;
     if (Nk % 8 != 0) return FA_ERR_UNSUPPORTED;  // bias rows are read in 16-byte chunks
@@ -159,6 +187,9 @@ fa_status make_ext(ExtArgs* ext, const void* bias, int bias_B, int bias_H, int B
     const long long plane = (long long)Nq * Nk;
     ext->sh = bias_H == 1 ? 0 : plane;
     ext->sb = bias_B == 1 ? 0 : (long long)bias_H * plane;
+    ext->ph = bias_H == 1 ? 0 : 1;
+    ext->pb = bias_B == 1 ? 0 : bias_H;
+    ext->planes = (long long)bias_B * bias_H;
   }
   return FA_OK;
 }
@@ -184,14 +215,23 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
   p.Nq = Nq;
   p.Nk = Nk;
   p.BH = BH;
-  // Two 128-row tiles per CTA (softmax / MMA ping-pong) unless that leaves SMs idle.
-  p.tiles = ((long long)((Nq + 255) / 256) * BH < num_sms()) ? 1 : 2;
+  // Two 128-row tiles per work item (softmax / MMA ping-pong) unless there are fewer such items than
+  // SMs; then one tile per item and one item per CTA.  With two tiles the grid is persistent: one CTA
+  // per SM walks its share of the items.
+  const int sms = num_sms();
+  p.tiles = ((long long)((Nq + 255) / 256) * BH < sms) ? 1 : 2;
   p.nunits = (Nq + 128 * p.tiles - 1) / (128 * p.tiles);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal ? 1 : 0;
-  const long long blocks = (long long)p.nunits * BH;
-  if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-  fa::fa_fwd_kernel<D, F8, EXT><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  const long long items = (long long)p.nunits * BH;
+  if (items > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+  const long long blocks = p.tiles == 2 ? (items < sms ? items : sms) : items;
+  // The kernel counts K/V loads per CTA in 32-bit integers.
+  const long long loads_per_cta = ((items + blocks - 1) / blocks) * 2LL * ((Nk + 127) / 128);
+  if (loads_per_cta > (1LL << 30)) return FA_ERR_UNSUPPORTED;
+  CUtensorMap mb;
+  if (!ext_bias_map(&mb, ext, Nq, Nk)) return FA_ERR_CUDA;
+  fa::fa_fwd_kernel<D, F8, EXT><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mb, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -234,11 +274,14 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.BH = BH;
     p.nkt = (Nk + 127) / 128;
     // Heads per group: their Q and dO (bf16) and dQ accumulator (fp32), 8 Nq d bytes a head,
-    // within ~32 MB of the 126 MB L2; at least 4 heads so that a group fills the SMs.
+    // within ~32 MB of the 126 MB L2, but at least enough heads for the group's key blocks to fill
+    // the SMs (one head of a long sequence already does).
     {
       const long long per_head = 8LL * Nq * D;
       long long g = (32LL << 20) / (per_head > 0 ? per_head : 1);
-      g = g < 4 ? 4 : g;
+      const long long fill = (num_sms() + p.nkt - 1) / p.nkt;
+      g = g < fill ? fill : g;
+      g = g < 1 ? 1 : g;
       p.hgroup = (int)(g < BH ? g : BH);
     }
     p.scale = scale;
@@ -246,13 +289,17 @@ fa_status launch_bwd(const void* q, const void* k, const void* v, const void* o,
     p.causal = causal ? 1 : 0;
     const long long blocks = (long long)p.nkt * BH;
     if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
+    CUtensorMap mb;
+    if (!ext_bias_map(&mb, ext, Nq, Nk)) return FA_ERR_CUDA;
     if (ext)
       fa::fa_bwd_main_kernel<D, true, true><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo,
-                                                                                                     mdq, p);
+                                                                                                     mdq, mb, p);
     else if (deterministic)
-      fa::fa_bwd_main_kernel<D, false><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
+      fa::fa_bwd_main_kernel<D, false><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq,
+                                                                                                mb, p);
     else
-      fa::fa_bwd_main_kernel<D, true><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq, p);
+      fa::fa_bwd_main_kernel<D, true><<<(unsigned)blocks, T::THREADS, T::SMEM_BYTES, stream>>>(mq, mk, mv, mdo, mdq,
+                                                                                               mb, p);
     if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
     if (deterministic && Nq > 0) {
       using TQ = fa::DqTraits<D>;

@@ -48,17 +48,22 @@ struct FwdTraits {
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128 x D tile
   static constexpr int KSTEP = 32 / EB;                // MMA K per instruction (32 bytes of operand)
   static constexpr int NS = F8 ? 8 : ((D == 64) ? 6 : 3);  // K/V ring stages
+  // Two Q slots (work items alternate between them, so the next item's Q loads while the current
+  // one runs), each holding the item's two 128-row tiles: slot s, tile t at OFF_Q + (2 s + t) TILE_BYTES.
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = 2 * TILE_BYTES;
+  static constexpr int OFF_KV = 4 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
-  // barriers: q_full | kv_full[NS] | kv_empty[NS] | s_full[2] | p_ready[2] | o_done[2] | drain
-  static constexpr int BAR_Q = 0;
-  static constexpr int BAR_KV_FULL = 1;
-  static constexpr int BAR_KV_EMPTY = 1 + NS;
-  static constexpr int BAR_S_FULL = 1 + 2 * NS;
+  // barriers: q_full[2] | q_empty[2] | kv_full[NS] | kv_empty[NS] | s_full[2] | p_ready[2] | o_done[2] |
+  //           o_free[2] | drain | merge
+  static constexpr int BAR_Q_FULL = 0;
+  static constexpr int BAR_Q_EMPTY = 2;
+  static constexpr int BAR_KV_FULL = 4;
+  static constexpr int BAR_KV_EMPTY = 4 + NS;
+  static constexpr int BAR_S_FULL = 4 + 2 * NS;
   static constexpr int BAR_P_READY = BAR_S_FULL + 2;
   static constexpr int BAR_O_DONE = BAR_P_READY + 2;
-  static constexpr int BAR_DRAIN = BAR_O_DONE + 2;
+  static constexpr int BAR_O_FREE = BAR_O_DONE + 2;  // group t has read O_t out: the next item may overwrite it
+  static constexpr int BAR_DRAIN = BAR_O_FREE + 2;
   static constexpr int BAR_MERGE = BAR_DRAIN + 1;  // split mode: group 1's row statistics published
   static constexpr int NBAR = BAR_MERGE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
@@ -77,8 +82,9 @@ struct FwdParams {
   float* lse;
   int Nq, Nk, BH;
   int nunits;        // query units per (batch, head): ceil(Nq / (128 * tiles))
-  int tiles;         // 128-row query tiles per CTA: 2 (ping-pong), or 1 when the grid would be small (then
-                     // the two softmax groups split that tile's key tiles: even / odd)
+  int tiles;         // 128-row query tiles per unit: 2 (ping-pong), or 1 when there are fewer units than
+                     // SMs (then each CTA takes one unit and the two softmax groups split its key tiles:
+                     // even / odd)
   float scale_log2;  // scale * log2(e)
   int causal;
   // FP8 operands only: per-(batch, head) dequantisation factors (x = x8 * descale).
@@ -86,11 +92,20 @@ struct FwdParams {
   const float* descale_k;
   const float* descale_v;
   // Bias and dropout instantiation only.  bias: [Bb, Hb, Nq, Nk] bf16 or null, b / h element
-  // strides bias_sb / bias_sh (0 where broadcast); H splits the (batch, head) index.
+  // strides bias_sb / bias_sh (0 where broadcast), and b / h strides bias_pb / bias_ph in [Nq, Nk]
+  // planes (the third coordinate of the bias tensor map); H splits the (batch, head) index.
   const __nv_bfloat16* bias;
   long long bias_sb, bias_sh;
+  int bias_pb, bias_ph;
   int H;
   DropoutCfg drop;
+};
+
+// One work item: the query unit of rows [q0, q0 + 128 tiles) of (batch, head) bh.  n0 / n1: key tiles
+// query tile 0 / 1 must visit (under the causal mask the last key tile of the unit is hidden from
+// tile 0 entirely, so tile 0 skips it); n_kv = max(n0, n1) K/V tiles are streamed.
+struct FwdItem {
+  int bh, q0, n0, n1, n_kv;
 };
 
 // Number of 128-key tiles the CTA owning query rows [q0, q0 + span) must visit.
@@ -184,7 +199,8 @@ __device__ __forceinline__ void fwd_apply_bias(float* s, const __nv_bfloat16* bi
 template <int D, bool F8 = false, bool EXT = false>
 __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
+                  const FwdParams p) {
   static_assert(!(F8 && EXT), "bias and dropout are not combined with FP8 operands");
   using T = FwdTraits<D, F8>;
   extern __shared__ uint8_t smem_raw[];
@@ -195,16 +211,39 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x % p.BH;
-  const int rank = blockIdx.x / p.BH;
-  const int unit = p.causal ? (p.nunits - 1 - rank) : rank;  // causal: heaviest tiles first
   const bool two = p.tiles == 2;
-  const int q0 = unit * 128 * p.tiles;
-  const int n_kv = fwd_num_kv_tiles(q0, 128 * p.tiles, p.Nq, p.Nk, p.causal);
-  int issued = 0;  // K/V loads started by the TMA producer (its lane 0), for the teardown
+  // Work items (query units of one (batch, head)), numbered heaviest first under the causal mask.
+  // A CTA takes one item per round of gridDim.x items, in a snake order over the CTAs (forward in
+  // even rounds, backward in odd ones), which evens out the causal work per CTA; with fewer items
+  // than CTAs (the split mode) every CTA has exactly one.  Every role walks the same list, and the
+  // K/V ring, the Q slots and all barrier phases run on across items.
+  const int n_items = p.nunits * p.BH;
+  const int G = gridDim.x;
+  auto item_at = [&](int r) -> int { return r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x); };
+  auto decode = [&](int i) -> FwdItem {
+    FwdItem w;
+    w.bh = i % p.BH;
+    const int rank = i / p.BH;
+    const int unit = p.causal ? (p.nunits - 1 - rank) : rank;
+    w.q0 = unit * 128 * p.tiles;
+    w.n0 = fwd_num_kv_tiles(w.q0, 128, p.Nq, p.Nk, p.causal);
+    w.n1 = two ? fwd_num_kv_tiles(w.q0 + 128, 128, p.Nq, p.Nk, p.causal) : w.n0;
+    w.n_kv = max(w.n0, w.n1);
+    return w;
+  };
+  int my_items = 0, total_loads = 0;
+  for (int r = 0; item_at(r) < n_items; ++r) {
+    ++my_items;
+    total_loads += 2 * decode(item_at(r)).n_kv;
+  }
+  int issued = 0;           // K/V loads started by the TMA producer (its lane 0), for the teardown
+  int q_fills[2] = {0, 0};  // Q loads per slot started by the TMA producer, for the teardown
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(T::BAR_Q), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(T::BAR_Q_FULL + s), 1);
+      mbar_init(bar(T::BAR_Q_EMPTY + s), 1);
+    }
     for (int s = 0; s < T::NS; ++s) {
       mbar_init(bar(T::BAR_KV_FULL + s), 1);
       mbar_init(bar(T::BAR_KV_EMPTY + s), 1);
@@ -213,6 +252,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
       mbar_init(bar(T::BAR_S_FULL + t), 1);
       mbar_init(bar(T::BAR_P_READY + t), 128);
       mbar_init(bar(T::BAR_O_DONE + t), 1);
+      mbar_init(bar(T::BAR_O_FREE + t), 128);
     }
     mbar_init(bar(T::BAR_DRAIN), 1);
     mbar_init(bar(T::BAR_MERGE), 128);
@@ -227,6 +267,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if (EXT && p.bias != nullptr) tma_prefetch_desc(&tmB);
   }
   tc_fence_before();
   __syncthreads();
@@ -235,299 +276,343 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
 
   if (warp < 8) {
     // ------------------------------------------------------------------ softmax warpgroups
-    // Two tiles: group t owns query tile t and visits every key tile.  Split (one query tile):
-    // group t visits key tiles t, t + 2, ... with its own running (m, l, O_t); group 0 merges.
+    // Two tiles: group t owns query tile t of each item.  Split (one query tile): group t visits
+    // the item's key tiles t, t + 2, ... with its own running (m, l, O_t); group 0 merges.
     const int t = warp >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // row in the tile == TMEM lane
-    const int row = q0 + (two ? 128 * t : 0) + r;  // query index within the head
-    const int n_own = two ? n_kv : (n_kv + 1 - t) / 2;  // key tiles this group visits
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
     const uint32_t colS = T::col_s(t), colO = T::col_o(t);
-    int kmax = p.Nk - 1;  // last visible key of this row (inclusive)
-    if (p.causal) kmax = min(kmax, row + p.Nk - p.Nq);
-    float m_run = -INFINITY, l_run = 0.f, lr_run = 0.f;
-    float scale_log2 = p.scale_log2;
-    if constexpr (F8) scale_log2 *= __ldg(p.descale_q + bh) * __ldg(p.descale_k + bh);
-    // EXT: the scores are turned into log2-domain logits s * scale * log2(e) + bias * log2(e) in
-    // place, so the exponent step below multiplies by 1.
-    const float2 sc2 = EXT ? make_float2(1.f, 1.f) : make_float2(scale_log2, scale_log2);
-    const __nv_bfloat16* bias_row = nullptr;
-    if constexpr (EXT) {
-      if (p.bias != nullptr && row < p.Nq)
-        bias_row = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + (size_t)row * p.Nk;
-    }
     bool ok = true;
-    for (int step = 0; step < n_own; ++step) {
-      const int j = two ? step : 2 * step + t;  // key tile
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL + t), step & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      // Load the S row in two halves; the second half's load overlaps the first half's max.
-      uint32_t sa[64], sb[64];
-      tmem_ld32x32b_x64_nowait(lane_addr + colS, sa);
-      tmem_wait_ld_x64(sa);
-      tmem_ld32x32b_x64_nowait(lane_addr + colS + 64, sb);
-      float* s = reinterpret_cast<float*>(sa);
-      float* s2 = reinterpret_cast<float*>(sb);
-      const int lim = kmax - 128 * j;  // keys [0, lim] of this tile are visible
-      const bool masked = __any_sync(0xffffffffu, lim < 127);
-      if (masked) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c > lim) s[c] = -INFINITY;
+    int cnt = 0;  // S tiles this group has processed in earlier items (barrier phases run on)
+    for (int it = 0; ok && item_at(it) < n_items; ++it) {
+      const FwdItem w = decode(item_at(it));
+      const int bh = w.bh;
+      const int row = w.q0 + (two ? 128 * t : 0) + r;  // query index within the head
+      const int n_own = two ? (t ? w.n1 : w.n0) : (w.n_kv + 1 - t) / 2;  // key tiles this group visits
+      int kmax = p.Nk - 1;  // last visible key of this row (inclusive)
+      if (p.causal) kmax = min(kmax, row + p.Nk - p.Nq);
+      float m_run = -INFINITY, l_run = 0.f, lr_run = 0.f;
+      float scale_log2 = p.scale_log2;
+      if constexpr (F8) scale_log2 *= __ldg(p.descale_q + bh) * __ldg(p.descale_k + bh);
+      // EXT: the scores are turned into log2-domain logits s * scale * log2(e) + bias * log2(e) in
+      // place, so the exponent step below multiplies by 1.
+      const float2 sc2 = EXT ? make_float2(1.f, 1.f) : make_float2(scale_log2, scale_log2);
+      const __nv_bfloat16* bias_row = nullptr;
+      if constexpr (EXT) {
+        if (p.bias != nullptr && row < p.Nq)
+          bias_row = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + (size_t)row * p.Nk;
       }
-      if constexpr (EXT) fwd_apply_bias(s, bias_row, 128 * j, p.Nk, scale_log2);
-      const float mx_a = max64(s);
-      tmem_wait_ld_x64(sb);
-      if (masked) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c + 64 > lim) s2[c] = -INFINITY;
-      }
-      if constexpr (EXT) fwd_apply_bias(s2, bias_row, 128 * j + 64, p.Nk, scale_log2);
-      const float mx = fmaxf(mx_a, max64(s2));
-      const float m_tile = EXT ? mx : mx * scale_log2;
-      float alpha = 1.f;
-      bool resc = false;
-      if (m_tile > m_run + kRescaleThreshold) {
-        alpha = ex2_approx(m_run - m_tile);
-        resc = (step > 0) && (m_run != -INFINITY);
-        m_run = m_tile;
-      }
-      const float base = (m_run == -INFINITY) ? 0.f : m_run;
-      const float2 nb2 = make_float2(-base, -base);
-      // Exponentials in four chunks of 16 pairs; each chunk of P (bf16 pairs) is stored to TMEM
-      // as soon as it is ready.  Two row sums: exact (for LSE) and of the rounded weights
-      // (normalises O so it stays a convex combination of V rows).
-      float2 sum_e[2], sum_r[2];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) sum_e[i] = sum_r[i] = make_float2(0.f, 0.f);
-      if constexpr (F8) {
-        // E4M3 weights, four per 32-bit column (P <= 2^8 stays inside the format's 448).
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const float* src = (ch < 2) ? s + 32 * ch : s2 + 32 * (ch - 2);
-          uint32_t pk[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float2 x0 = ffma2(make_float2(src[4 * c], src[4 * c + 1]), sc2, nb2);
-            const float2 x1 = ffma2(make_float2(src[4 * c + 2], src[4 * c + 3]), sc2, nb2);
-            const float2 e0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
-            const float2 e1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
-            const uint32_t lo = f32x2_to_e4m3x2(e0.x, e0.y), hi = f32x2_to_e4m3x2(e1.x, e1.y);
-            pk[c] = lo | (hi << 16);
-            sum_e[0] = fadd2(sum_e[0], e0);
-            sum_e[1] = fadd2(sum_e[1], e1);
-            sum_r[0] = fadd2(sum_r[0], e4m3x2_to_f32x2(lo));
-            sum_r[1] = fadd2(sum_r[1], e4m3x2_to_f32x2(hi));
-          }
-          tmem_st32x32b_x8(lane_addr + colS + 8 * ch, pk);
-        }
-      } else {
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const float* src = (ch < 2) ? s + 32 * ch : s2 + 32 * (ch - 2);
-          uint32_t pk[16];
-          uint32_t keep[8];  // EXT with dropout: 0xff per kept key of this chunk's 8 key quads
-          if constexpr (EXT) {
-            if (p.drop.p8 != 0) dropout_keep_rowwise(p.drop, (uint32_t)(32 * j + 8 * ch), (uint32_t)row, (uint32_t)bh,
-                                                     lane, keep);
-          }
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float2 x = ffma2(make_float2(src[2 * c], src[2 * c + 1]), sc2, nb2);
-            const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            pk[c] = pack_bf16x2(e.x, e.y);
-            sum_e[c & 1] = fadd2(sum_e[c & 1], e);
-            sum_r[c & 1] = fadd2(sum_r[c & 1], make_float2(bf16lo_to_f32(pk[c]), bf16hi_to_f32(pk[c])));
-            if constexpr (EXT) {
-              // Dropped weights leave the normalising sums untouched and enter P V as +0.
-              if (p.drop.p8 != 0) pk[c] &= __byte_perm(keep[c >> 1], 0u, (c & 1) ? 0x3322u : 0x1100u);
-            }
-          }
-          tmem_st32x32b_x16(lane_addr + colS + 16 * ch, pk);
-        }
-      }
-      const float2 tot_e = fadd2(sum_e[0], sum_e[1]);
-      const float2 tot_r = fadd2(sum_r[0], sum_r[1]);
-      l_run = l_run * alpha + (tot_e.x + tot_e.y);
-      lr_run = lr_run * alpha + (tot_r.x + tot_r.y);
-      if (__any_sync(0xffffffffu, resc)) {
-        // O_t still holds the sum through this group's previous tile: wait until that PV has
-        // landed, then scale.
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (step - 1) & 1, abort_flag));
+      for (int step = 0; step < n_own; ++step) {
+        const int j = two ? step : 2 * step + t;  // key tile
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL + t), (cnt + step) & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
+        // Load the S row in two halves; the second half's load overlaps the first half's max.
+        uint32_t sa[64], sb[64];
+        tmem_ld32x32b_x64_nowait(lane_addr + colS, sa);
+        tmem_wait_ld_x64(sa);
+        tmem_ld32x32b_x64_nowait(lane_addr + colS + 64, sb);
+        float* s = reinterpret_cast<float*>(sa);
+        float* s2 = reinterpret_cast<float*>(sb);
+        const int lim = kmax - 128 * j;  // keys [0, lim] of this tile are visible
+        const bool masked = __any_sync(0xffffffffu, lim < 127);
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c > lim) s[c] = -INFINITY;
+        }
+        if constexpr (EXT) fwd_apply_bias(s, bias_row, 128 * j, p.Nk, scale_log2);
+        const float mx_a = max64(s);
+        tmem_wait_ld_x64(sb);
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c + 64 > lim) s2[c] = -INFINITY;
+        }
+        if constexpr (EXT) fwd_apply_bias(s2, bias_row, 128 * j + 64, p.Nk, scale_log2);
+        const float mx = fmaxf(mx_a, max64(s2));
+        const float m_tile = EXT ? mx : mx * scale_log2;
+        float alpha = 1.f;
+        bool resc = false;
+        if (m_tile > m_run + kRescaleThreshold) {
+          alpha = ex2_approx(m_run - m_tile);
+          resc = (step > 0) && (m_run != -INFINITY);
+          m_run = m_tile;
+        }
+        const float base = (m_run == -INFINITY) ? 0.f : m_run;
+        const float2 nb2 = make_float2(-base, -base);
+        // Exponentials in four chunks of 16 pairs; each chunk of P (bf16 pairs) is stored to TMEM
+        // as soon as it is ready.  Two row sums: exact (for LSE) and of the rounded weights
+        // (normalises O so it stays a convex combination of V rows).
+        float2 sum_e[2], sum_r[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) sum_e[i] = sum_r[i] = make_float2(0.f, 0.f);
+        if constexpr (F8) {
+          // E4M3 weights, four per 32-bit column (P <= 2^8 stays inside the format's 448).
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const float* src = (ch < 2) ? s + 32 * ch : s2 + 32 * (ch - 2);
+            uint32_t pk[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float2 x0 = ffma2(make_float2(src[4 * c], src[4 * c + 1]), sc2, nb2);
+              const float2 x1 = ffma2(make_float2(src[4 * c + 2], src[4 * c + 3]), sc2, nb2);
+              const float2 e0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+              const float2 e1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+              const uint32_t lo = f32x2_to_e4m3x2(e0.x, e0.y), hi = f32x2_to_e4m3x2(e1.x, e1.y);
+              pk[c] = lo | (hi << 16);
+              sum_e[0] = fadd2(sum_e[0], e0);
+              sum_e[1] = fadd2(sum_e[1], e1);
+              sum_r[0] = fadd2(sum_r[0], e4m3x2_to_f32x2(lo));
+              sum_r[1] = fadd2(sum_r[1], e4m3x2_to_f32x2(hi));
+            }
+            tmem_st32x32b_x8(lane_addr + colS + 8 * ch, pk);
+          }
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const float* src = (ch < 2) ? s + 32 * ch : s2 + 32 * (ch - 2);
+            uint32_t pk[16];
+            uint32_t keep[8];  // EXT with dropout: 0xff per kept key of this chunk's 8 key quads
+            if constexpr (EXT) {
+              if (p.drop.p8 != 0)
+                dropout_keep_rowwise(p.drop, (uint32_t)(32 * j + 8 * ch), (uint32_t)row, (uint32_t)bh, lane, keep);
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              const float2 x = ffma2(make_float2(src[2 * c], src[2 * c + 1]), sc2, nb2);
+              const float2 e = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+              pk[c] = pack_bf16x2(e.x, e.y);
+              sum_e[c & 1] = fadd2(sum_e[c & 1], e);
+              sum_r[c & 1] = fadd2(sum_r[c & 1], make_float2(bf16lo_to_f32(pk[c]), bf16hi_to_f32(pk[c])));
+              if constexpr (EXT) {
+                // Dropped weights leave the normalising sums untouched and enter P V as +0.
+                if (p.drop.p8 != 0) pk[c] &= __byte_perm(keep[c >> 1], 0u, (c & 1) ? 0x3322u : 0x1100u);
+              }
+            }
+            tmem_st32x32b_x16(lane_addr + colS + 16 * ch, pk);
+          }
+        }
+        const float2 tot_e = fadd2(sum_e[0], sum_e[1]);
+        const float2 tot_r = fadd2(sum_r[0], sum_r[1]);
+        l_run = l_run * alpha + (tot_e.x + tot_e.y);
+        lr_run = lr_run * alpha + (tot_r.x + tot_r.y);
+        if (__any_sync(0xffffffffu, resc)) {
+          // O_t still holds the sum through this group's previous tile: wait until that PV has
+          // landed, then scale.
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (cnt + step - 1) & 1, abort_flag));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32x32b_x32_wait(lane_addr + colO + 32 * c, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32x32b_x32(lane_addr + colO + 32 * c, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(T::BAR_P_READY + t));
+      }
+      if (!ok) break;
+      // This group's accumulator is complete once its last PV has landed.
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (cnt + n_own - 1) & 1, abort_flag));
+      cnt += n_own;
+      float* merge_stats = reinterpret_cast<float*>(smem + T::OFF_Q + T::TILE_BYTES);  // split: slot 0 tile 1 unused
+      if (ok && !two && t == 1) {
+        // Split: publish (m, l, l of the rounded weights) for group 0, which merges both halves.
+        merge_stats[r] = m_run;
+        merge_stats[128 + r] = l_run;
+        merge_stats[256 + r] = lr_run;
+        mbar_arrive(bar(T::BAR_MERGE));
+      }
+      // Weights of O_0 and O_1 in the merged sum: the two-block identity of the online softmax (each
+      // group's sums are relative to its own running maximum).
+      float a0 = 1.f, a1 = 0.f;
+      bool use1 = false;
+      if (ok && !two && t == 0) {
+        // Split (one item per CTA): group 1's statistics and (if it visited any key tile) its
+        // accumulator.
+        const int n1 = w.n_kv / 2;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_MERGE), 0, abort_flag));
+        if (ok && n1 > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + 1), (n1 - 1) & 1, abort_flag));
+        if (ok) {
+          const float m1 = merge_stats[r], l1 = merge_stats[128 + r], lr1 = merge_stats[256 + r];
+          const float m = fmaxf(m_run, m1);
+          a0 = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m);
+          a1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - m);
+          l_run = a0 * l_run + a1 * l1;
+          lr_run = a0 * lr_run + a1 * lr1;
+          m_run = m;
+          use1 = n1 > 0;
+        }
+      }
+      if (ok && (two || t == 0)) {
+        tc_fence_after();
+        float num = 1.f;
+        if constexpr (F8) num = __ldg(p.descale_v + bh);
+        if constexpr (EXT) num = p.drop.scale;
+        const float inv = lr_run > 0.f ? num / lr_run : 0.f;
+        const bool in_range = row < p.Nq;
+        __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
           tmem_ld32x32b_x32_wait(lane_addr + colO + 32 * c, o);
+          if (use1) {
+            uint32_t o1[32];
+            tmem_ld32x32b_x32_wait(lane_addr + T::col_o(1) + 32 * c, o1);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32x32b_x32(lane_addr + colO + 32 * c, o);
+            for (int i = 0; i < 32; ++i)
+              o[i] = __float_as_uint(a0 * __uint_as_float(o[i]) + a1 * __uint_as_float(o1[i]));
+          } else if (!two) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(a0 * __uint_as_float(o[i]));
+          }
+          uint32_t wv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            wv[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+          if (in_range) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
+          }
         }
+        // O_t is in registers and on its way out: the next item's first P V may overwrite it.
+        tc_fence_before();
+        mbar_arrive(bar(T::BAR_O_FREE + t));
+        if (in_range) p.lse[(size_t)bh * p.Nq + row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(T::BAR_P_READY + t));
-    }
-    // This group's accumulator is complete once its last PV has landed.
-    if (ok && n_own > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (n_own - 1) & 1, abort_flag));
-    float* merge_stats = reinterpret_cast<float*>(smem + T::OFF_Q + T::TILE_BYTES);  // split: Q slot 1 unused
-    if (ok && !two && t == 1) {
-      // Split: publish (m, l, l of the rounded weights) for group 0, which merges both halves.
-      merge_stats[r] = m_run;
-      merge_stats[128 + r] = l_run;
-      merge_stats[256 + r] = lr_run;
-      mbar_arrive(bar(T::BAR_MERGE));
-    }
-    // Weights of O_0 and O_1 in the merged sum: the two-block identity of the online softmax (each
-    // group's sums are relative to its own running maximum).
-    float a0 = 1.f, a1 = 0.f;
-    bool use1 = false;
-    if (ok && !two && t == 0) {
-      // Split: group 1's statistics and (if it visited any key tile) its accumulator.
-      const int n1 = n_kv / 2;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_MERGE), 0, abort_flag));
-      if (ok && n1 > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + 1), (n1 - 1) & 1, abort_flag));
-      if (ok) {
-        const float m1 = merge_stats[r], l1 = merge_stats[128 + r], lr1 = merge_stats[256 + r];
-        const float m = fmaxf(m_run, m1);
-        a0 = (m_run == -INFINITY) ? 0.f : ex2_approx(m_run - m);
-        a1 = (m1 == -INFINITY) ? 0.f : ex2_approx(m1 - m);
-        l_run = a0 * l_run + a1 * l1;
-        lr_run = a0 * lr_run + a1 * lr1;
-        m_run = m;
-        use1 = n1 > 0;
-      }
-    }
-    if (ok && (two || t == 0)) {
-      tc_fence_after();
-      float num = 1.f;
-      if constexpr (F8) num = __ldg(p.descale_v + bh);
-      if constexpr (EXT) num = p.drop.scale;
-      const float inv = lr_run > 0.f ? num / lr_run : 0.f;
-      const bool in_range = row < p.Nq;
-      __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32x32b_x32_wait(lane_addr + colO + 32 * c, o);
-        if (use1) {
-          uint32_t o1[32];
-          tmem_ld32x32b_x32_wait(lane_addr + T::col_o(1) + 32 * c, o1);
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            o[i] = __float_as_uint(a0 * __uint_as_float(o[i]) + a1 * __uint_as_float(o1[i]));
-        } else if (!two) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(a0 * __uint_as_float(o[i]));
-        }
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-        if (in_range) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-        }
-      }
-      if (in_range) p.lse[(size_t)bh * p.Nq + row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
     }
     if (!ok) *abort_flag = 1;
   } else if (warp == 8) {
     // ------------------------------------------------------------------ MMA issuer
     {  // the whole warp, converged: one elected lane issues
-      const int total_loads = 2 * n_kv;
       auto release = [&](int load_idx) {
         // Only stages the producer will refill get an "empty" arrival.
         if (load_idx + T::NS < total_loads) mma_commit_w(bar(T::BAR_KV_EMPTY + load_idx % T::NS));
       };
-      const uint32_t q_smem[2] = {sbase + T::OFF_Q, sbase + T::OFF_Q + T::TILE_BYTES};
+      auto kv_smem = [&](int load_idx) { return sbase + T::OFF_KV + (load_idx % T::NS) * T::TILE_BYTES; };
+      auto kv_wait = [&](int load_idx) {
+        return warp_wait(bar(T::BAR_KV_FULL + load_idx % T::NS), (load_idx / T::NS) & 1, abort_flag);
+      };
       const uint32_t tS[2] = {tmem_base + T::col_s(0), tmem_base + T::col_s(1)};
       const uint32_t tO[2] = {tmem_base + T::col_o(0), tmem_base + T::col_o(1)};
-      bool ok = warp_wait(bar(T::BAR_Q), 0, abort_flag);
-      int v_prev = -1;
-      if (!two) {
-        // Split: step i computes S_0 = Q K(2i)^T and S_1 = Q K(2i+1)^T, then O_0 += P_0 V(2i) and
-        // (one step later, like the two-tile order) O_1 += P_1 V(2i+1).  Loads arrive in the ring
-        // order K(j), V(j), K(j+1), V(j+1), ...
-        const int nsteps = (n_kv + 1) / 2;
-        int v1_prev = -1;  // load index of the V tile of group 1's pending PV
-        for (int i = 0; ok && i < nsteps; ++i) {
-          const int ik0 = 4 * i, iv0 = 4 * i + 1, ik1 = 4 * i + 2, iv1 = 4 * i + 3;
-          const bool has1 = 2 * i + 1 < n_kv;
-          if (!(ok = warp_wait(bar(T::BAR_KV_FULL + ik0 % T::NS), (ik0 / T::NS) & 1, abort_flag))) break;
-          tc_fence_after();
-          fwd_issue_qk<D, F8>(tS[0], q_smem[0], sbase + T::OFF_KV + (ik0 % T::NS) * T::TILE_BYTES);
-          mma_commit_w(bar(T::BAR_S_FULL + 0));
-          release(ik0);
-          if (v1_prev >= 0) {
-            if (!(ok = warp_wait(bar(T::BAR_KV_FULL + v1_prev % T::NS), (v1_prev / T::NS) & 1, abort_flag))) break;
-            if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (i - 1) & 1, abort_flag))) break;
+      bool ok = true;
+      int L = 0;                // global index of the item's first K/V load
+      int cnt0 = 0, cnt1 = 0;   // S tiles of groups 0 / 1 in earlier items (barrier phases run on)
+      for (int k = 0; ok && item_at(k) < n_items; ++k) {
+        const FwdItem w = decode(item_at(k));
+        const int slot = k & 1;
+        const uint32_t q_smem[2] = {sbase + T::OFF_Q + (2 * slot) * T::TILE_BYTES,
+                                    sbase + T::OFF_Q + (2 * slot + 1) * T::TILE_BYTES};
+        if (!(ok = warp_wait(bar(T::BAR_Q_FULL + slot), (k >> 1) & 1, abort_flag))) break;
+        // The first P V of group t in this item overwrites O_t: group t must have read out the
+        // previous item's output (two-tile mode; the split mode has one item per CTA).
+        auto o_free = [&](int t) {
+          return k == 0 || warp_wait(bar(T::BAR_O_FREE + t), (k - 1) & 1, abort_flag);
+        };
+        if (!two) {
+          // Split: step i computes S_0 = Q K(2i)^T and S_1 = Q K(2i+1)^T, then O_0 += P_0 V(2i) and
+          // (one step later, like the two-tile order) O_1 += P_1 V(2i+1).  Loads arrive in the ring
+          // order K(j), V(j), K(j+1), V(j+1), ...
+          const int n_kv = w.n_kv;
+          const int nsteps = (n_kv + 1) / 2;
+          int v1_prev = -1;  // load index of the V tile of group 1's pending PV
+          for (int i = 0; ok && i < nsteps; ++i) {
+            const int ik0 = L + 4 * i, iv0 = ik0 + 1, ik1 = ik0 + 2, iv1 = ik0 + 3;
+            const bool has1 = 2 * i + 1 < n_kv;
+            if (!(ok = kv_wait(ik0))) break;
             tc_fence_after();
-            fwd_issue_pv<D, F8>(tO[1], tS[1], sbase + T::OFF_KV + (v1_prev % T::NS) * T::TILE_BYTES, i - 1 > 0);
-            mma_commit_w(bar(T::BAR_O_DONE + 1));
-            release(v1_prev);
-            v1_prev = -1;
+            fwd_issue_qk<D, F8>(tS[0], q_smem[0], kv_smem(ik0));
+            mma_commit_w(bar(T::BAR_S_FULL + 0));
+            release(ik0);
+            if (v1_prev >= 0) {
+              if (!(ok = kv_wait(v1_prev))) break;
+              if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (cnt1 + i - 1) & 1, abort_flag))) break;
+              tc_fence_after();
+              fwd_issue_pv<D, F8>(tO[1], tS[1], kv_smem(v1_prev), i - 1 > 0);
+              mma_commit_w(bar(T::BAR_O_DONE + 1));
+              release(v1_prev);
+              v1_prev = -1;
+            }
+            if (has1) {
+              if (!(ok = kv_wait(ik1))) break;
+              tc_fence_after();
+              fwd_issue_qk<D, F8>(tS[1], q_smem[0], kv_smem(ik1));
+              mma_commit_w(bar(T::BAR_S_FULL + 1));
+              release(ik1);
+              v1_prev = iv1;
+            }
+            if (!(ok = kv_wait(iv0))) break;
+            if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), (cnt0 + i) & 1, abort_flag))) break;
+            tc_fence_after();
+            fwd_issue_pv<D, F8>(tO[0], tS[0], kv_smem(iv0), i > 0);
+            mma_commit_w(bar(T::BAR_O_DONE + 0));
+            release(iv0);
           }
-          if (has1) {
-            if (!(ok = warp_wait(bar(T::BAR_KV_FULL + ik1 % T::NS), (ik1 / T::NS) & 1, abort_flag))) break;
+          if (ok && v1_prev >= 0) {
+            const int i = nsteps - 1;
+            if ((ok = kv_wait(v1_prev)) && (ok = warp_wait(bar(T::BAR_P_READY + 1), (cnt1 + i) & 1, abort_flag))) {
+              tc_fence_after();
+              fwd_issue_pv<D, F8>(tO[1], tS[1], kv_smem(v1_prev), i > 0);
+              mma_commit_w(bar(T::BAR_O_DONE + 1));
+              release(v1_prev);
+            }
+          }
+          cnt0 += (n_kv + 1) / 2;
+          cnt1 += n_kv / 2;
+        } else {
+          // Two tiles, in the order S0 S1 PV0 S0' PV1 S1' ...; query tile 0 skips the key tiles it
+          // cannot see (j >= n0), tile 1 visits all n_kv = n1.
+          int v_prev = -1;
+          for (int j = 0; ok && j < w.n_kv; ++j) {
+            const int ik = L + 2 * j, iv = ik + 1;
+            if (!(ok = kv_wait(ik))) break;
             tc_fence_after();
-            fwd_issue_qk<D, F8>(tS[1], q_smem[0], sbase + T::OFF_KV + (ik1 % T::NS) * T::TILE_BYTES);
+            if (j < w.n0) {
+              fwd_issue_qk<D, F8>(tS[0], q_smem[0], kv_smem(ik));
+              mma_commit_w(bar(T::BAR_S_FULL + 0));
+            }
+            if (j > 0) {
+              if (j == 1 && !(ok = o_free(1))) break;
+              if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (cnt1 + j - 1) & 1, abort_flag))) break;
+              tc_fence_after();
+              fwd_issue_pv<D, F8>(tO[1], tS[1], kv_smem(v_prev), j - 1 > 0);
+              mma_commit_w(bar(T::BAR_O_DONE + 1));
+              release(v_prev);
+            }
+            fwd_issue_qk<D, F8>(tS[1], q_smem[1], kv_smem(ik));
             mma_commit_w(bar(T::BAR_S_FULL + 1));
-            release(ik1);
-            v1_prev = iv1;
+            release(ik);
+            if (!(ok = kv_wait(iv))) break;
+            if (j < w.n0) {
+              if (j == 0 && !(ok = o_free(0))) break;
+              if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), (cnt0 + j) & 1, abort_flag))) break;
+              tc_fence_after();
+              fwd_issue_pv<D, F8>(tO[0], tS[0], kv_smem(iv), j > 0);
+              mma_commit_w(bar(T::BAR_O_DONE + 0));
+            }
+            v_prev = iv;
           }
-          if (!(ok = warp_wait(bar(T::BAR_KV_FULL + iv0 % T::NS), (iv0 / T::NS) & 1, abort_flag))) break;
-          if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), i & 1, abort_flag))) break;
-          tc_fence_after();
-          fwd_issue_pv<D, F8>(tO[0], tS[0], sbase + T::OFF_KV + (iv0 % T::NS) * T::TILE_BYTES, i > 0);
-          mma_commit_w(bar(T::BAR_O_DONE + 0));
-          release(iv0);
-        }
-        if (ok && v1_prev >= 0) {
-          const int i = nsteps - 1;
-          if ((ok = warp_wait(bar(T::BAR_KV_FULL + v1_prev % T::NS), (v1_prev / T::NS) & 1, abort_flag)) &&
-              (ok = warp_wait(bar(T::BAR_P_READY + 1), i & 1, abort_flag))) {
+          if (ok && w.n_kv == 1) ok = o_free(1);
+          if (ok && (ok = warp_wait(bar(T::BAR_P_READY + 1), (cnt1 + w.n_kv - 1) & 1, abort_flag))) {
             tc_fence_after();
-            fwd_issue_pv<D, F8>(tO[1], tS[1], sbase + T::OFF_KV + (v1_prev % T::NS) * T::TILE_BYTES, i > 0);
+            fwd_issue_pv<D, F8>(tO[1], tS[1], kv_smem(v_prev), w.n_kv - 1 > 0);
             mma_commit_w(bar(T::BAR_O_DONE + 1));
+            release(v_prev);
           }
+          cnt0 += w.n0;
+          cnt1 += w.n1;
         }
-      }
-      for (int j = 0; two && ok && j < n_kv; ++j) {
-        const int ik = 2 * j, iv = 2 * j + 1;
-        const int sk = ik % T::NS, sv = iv % T::NS;
-        const uint32_t k_smem = sbase + T::OFF_KV + sk * T::TILE_BYTES;
-        const uint32_t v_smem = sbase + T::OFF_KV + sv * T::TILE_BYTES;
-        if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sk), (ik / T::NS) & 1, abort_flag))) break;
-        tc_fence_after();
-        fwd_issue_qk<D, F8>(tS[0], q_smem[0], k_smem);
-        mma_commit_w(bar(T::BAR_S_FULL + 0));
-        if (j > 0) {
-          if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (j - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          fwd_issue_pv<D, F8>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, j - 1 > 0);
-          mma_commit_w(bar(T::BAR_O_DONE + 1));
-          release(v_prev);
-        }
-        fwd_issue_qk<D, F8>(tS[1], q_smem[1], k_smem);
-        mma_commit_w(bar(T::BAR_S_FULL + 1));
-        release(ik);
-        if (!(ok = warp_wait(bar(T::BAR_KV_FULL + sv), (iv / T::NS) & 1, abort_flag))) break;
-        if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), j & 1, abort_flag))) break;
-        tc_fence_after();
-        fwd_issue_pv<D, F8>(tO[0], tS[0], v_smem, j > 0);
-        mma_commit_w(bar(T::BAR_O_DONE + 0));
-        v_prev = iv;
-      }
-      if (two && ok && (ok = warp_wait(bar(T::BAR_P_READY + 1), (n_kv - 1) & 1, abort_flag))) {
-        tc_fence_after();
-        fwd_issue_pv<D, F8>(tO[1], tS[1], sbase + T::OFF_KV + (v_prev % T::NS) * T::TILE_BYTES, n_kv - 1 > 0);
-        mma_commit_w(bar(T::BAR_O_DONE + 1));
+        // Every S MMA of this item has been issued: its Q slot is free once they complete (the
+        // commit tracks all earlier MMAs of this thread).  Only slots the producer refills.
+        if (ok && k + 2 < my_items) mma_commit_w(bar(T::BAR_Q_EMPTY + slot));
+        L += 2 * w.n_kv;
       }
       if (!ok) *abort_flag = 1;
     }
@@ -535,22 +620,40 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
   } else {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(T::BAR_Q), p.tiles * T::TILE_BYTES);
-      for (int t = 0; t < p.tiles; ++t)
-        for (int b = 0; b < T::NBOX; ++b)
-          tma_load_3d(sbase + T::OFF_Q + t * T::TILE_BYTES + b * T::BOX_BYTES, &tmQ, bar(T::BAR_Q), T::BOX_COLS * b,
-                      q0 + 128 * t, bh);
-      const int total_loads = 2 * n_kv;
       bool ok = true;
-      for (int idx = 0; idx < total_loads; ++idx) {
-        const int s = idx % T::NS;
-        if (!(ok = mbar_wait(bar(T::BAR_KV_EMPTY + s), ((idx / T::NS) & 1) ^ 1, abort_flag))) break;
-        mbar_arrive_expect_tx(bar(T::BAR_KV_FULL + s), T::TILE_BYTES);
-        const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
-        for (int b = 0; b < T::NBOX; ++b)
-          tma_load_3d(sbase + T::OFF_KV + s * T::TILE_BYTES + b * T::BOX_BYTES, map, bar(T::BAR_KV_FULL + s),
-                      T::BOX_COLS * b, 128 * (idx >> 1), bh);
-        issued = idx + 1;
+      int L = 0;  // global index of the item's first K/V load
+      for (int k = 0; ok && item_at(k) < n_items; ++k) {
+        const FwdItem w = decode(item_at(k));
+        const int slot = k & 1;
+        // The slot's previous item (k - 2) must have finished its S MMAs.
+        if (k >= 2 && !(ok = mbar_wait(bar(T::BAR_Q_EMPTY + slot), ((k - 2) >> 1) & 1, abort_flag))) break;
+        mbar_arrive_expect_tx(bar(T::BAR_Q_FULL + slot), p.tiles * T::TILE_BYTES);
+        for (int t = 0; t < p.tiles; ++t)
+          for (int b = 0; b < T::NBOX; ++b)
+            tma_load_3d(sbase + T::OFF_Q + (2 * slot + t) * T::TILE_BYTES + b * T::BOX_BYTES, &tmQ,
+                        bar(T::BAR_Q_FULL + slot), T::BOX_COLS * b, w.q0 + 128 * t, w.bh);
+        ++q_fills[slot];
+        for (int idx = 0; idx < 2 * w.n_kv; ++idx) {
+          const int g = L + idx;
+          const int s = g % T::NS;
+          if (!(ok = mbar_wait(bar(T::BAR_KV_EMPTY + s), ((g / T::NS) & 1) ^ 1, abort_flag))) break;
+          mbar_arrive_expect_tx(bar(T::BAR_KV_FULL + s), T::TILE_BYTES);
+          const CUtensorMap* map = (idx & 1) ? &tmV : &tmK;
+          for (int b = 0; b < T::NBOX; ++b)
+            tma_load_3d(sbase + T::OFF_KV + s * T::TILE_BYTES + b * T::BOX_BYTES, map, bar(T::BAR_KV_FULL + s),
+                        T::BOX_COLS * b, 128 * (idx >> 1), w.bh);
+          issued = g + 1;
+          if constexpr (EXT) {
+            // Warm the L2 with the bias tiles of this key tile (each softmax row reads its 256 bytes
+            // with plain loads about NS loads later).
+            if (p.bias != nullptr && !(idx & 1)) {
+              const int plane = (w.bh / p.H) * p.bias_pb + (w.bh % p.H) * p.bias_ph;
+              for (int t = 0; t < p.tiles; ++t)
+                for (int b = 0; b < 2; ++b) tma_prefetch_l2_3d(&tmB, 128 * (idx >> 1) + 64 * b, w.q0 + 128 * t, plane);
+            }
+          }
+        }
+        L += 2 * w.n_kv;
       }
       if (!ok) *abort_flag = 1;
     }
@@ -575,7 +678,8 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
   } else if (warp == 9 && lane == 0 && aborted) {
     for (int idx = max(0, issued - T::NS); idx < issued; ++idx)
       drain_wait(bar(T::BAR_KV_FULL + idx % T::NS), (idx / T::NS) & 1);
-    drain_wait(bar(T::BAR_Q), 0);
+    for (int slot = 0; slot < 2; ++slot)
+      if (q_fills[slot] > 0) drain_wait(bar(T::BAR_Q_FULL + slot), (q_fills[slot] - 1) & 1);
   }
 }
 

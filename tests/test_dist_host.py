@@ -67,8 +67,8 @@ def test_measured_peaks_read():
     assert p["bf16_tflops"] > 100 and p["hbm_gbs"] > 1000
 
 
-def test_long_context_measurement_host_logic():
-    """bench.py's long-context block with a stand-in for the library (no GPU call): it allocates the
+def test_attn_point_host_logic():
+    """bench.py's per-workload block with a stand-in for the library (no GPU call): it allocates the
     right shapes and turns times into the FLOP-rate fields."""
     import types
 
@@ -85,10 +85,39 @@ def test_long_context_measurement_host_logic():
         fa_bwd=lambda *a: calls.append("bwd"),
         fa_get_device_error=lambda stream: 0)
     small = W.AttnConfig("long_small", 1, 2, 256, 256, 128, (True,), seed=3, peaked_frac=0.01)
-    out = bench.long_context_measurement(fake, W, torch.device("cpu"), None, {"bf16_tflops": 1000.0},
-                                         lambda fn: (fn(), 1e-3)[1], cfg=small)
+    out = bench.attn_point(fake, W, torch.device("cpu"), None, {"bf16_tflops": 1000.0},
+                           lambda fn: (fn(), 1e-3)[1], small)
     assert calls == ["fwd", "bwd"]
     ff = W.flops_forward(1, 2, 256, 256, 128, True)
     assert abs(out["fwd_tflops"] - ff / 1e-3 / 1e12) < 1e-12
     assert abs(out["fwd_bwd_tflops"] - 3.5 * ff / 2e-3 / 1e12) < 1e-12
     assert out["device_status"] == 0 and out["N"] == 256
+
+
+def test_visible_pairs_and_cpu_sample_flops():
+    """The CPU baseline counts FLOPs over the visible (query, key) pairs of its row blocks: summed over
+    all blocks that is N (N + 1) / 2 pairs under the causal mask (the convention's N^2 / 2, up to N / 2)."""
+    import bench
+    from io_aware_exact_32_b200 import workloads as W
+    n = 1024
+    assert sum(bench.visible_keys(r, r + 256, n, n, True) for r in range(0, n, 256)) == n * (n + 1) // 2
+    assert bench.visible_keys(0, 4, 10, 10, False) == 40
+    assert bench.visible_keys(0, 3, 5, 3, True) == 0 + 0 + 1      # bottom-right: rows 0, 1 see nothing
+    cfg = W.AttnConfig("t", 1, 1, 512, 512, 64, (True,), seed=0)
+    x = W.make_config_inputs(cfg)
+    flops, el, nblk, _ = bench.cpu_oracle_blocks(0.0, cfg, x, steps=2)
+    assert nblk == 2 and el > 0
+    want = sum(3.5 * 4 * 64 * bench.visible_keys(r0, r0 + 256, 512, 512, True)
+               for r0 in ((0 * 7919) % 2 * 256, (1 * 7919) % 2 * 256))
+    assert flops == want
+
+
+def test_clock_summary():
+    import bench
+    rows = ["0, 1965, 1965, 700.5, 0x0, Not Active, Not Active, Not Active, Not Active",
+            "0, 1800, 1965, 990.1, 0x4, Not Active, Not Active, Not Active, Active",
+            "0, 300, 1965, 100.0, 0x0, Not Active, Not Active, Not Active, Not Active"]
+    s = bench.summarize_clocks(rows)
+    assert s["sm_mhz"] == (1965 + 1800) / 2 and s["sm_max_mhz"] == 1965 and s["reasons"] == ["sw_power_cap"]
+    assert s["samples"] == 3
+    assert bench.summarize_clocks([])["reasons"] == ["unsampled"]

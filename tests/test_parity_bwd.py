@@ -54,6 +54,8 @@ RAGGED = [
     (1, 2, 384, 640, 64, False),
     (3, 2, 256, 256, 128, True),
     (1, 1, 513, 1025, 128, True),
+    (2, 40, 700, 1300, 128, True),
+    (2, 40, 1300, 700, 64, True),
 ]
 
 

@@ -50,6 +50,12 @@ RAGGED = [
     (1, 2, 384, 640, 64, False),
     (3, 2, 256, 256, 128, True),
     (1, 1, 513, 1025, 128, True),
+    # Enough 256-row units for the persistent two-tile grid (several units per CTA): Nq < Nk, Nq > Nk
+    # (whole units whose rows see no key), and a last unit whose second tile lies past Nq.
+    (2, 40, 700, 1300, 128, True),
+    (2, 40, 1300, 700, 64, True),
+    (1, 160, 300, 300, 128, False),
+    (1, 160, 300, 300, 64, True),
 ]
 
 
