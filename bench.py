@@ -621,7 +621,8 @@ def small_step(fa, W, dev, stream, peaks, flush_buf, reps=200):
 
 
 CASES = ("fwd_c2", "bwd_c2", "fwd_n4096_d128", "bwd_n4096_d128", "fwd_fp8_n4096_d128", "fwd_ext_n4096_d128",
-         "bwd_ext_n4096_d128", "decode", "fwd_long", "bwd_long", "bwd_n16384_d128", "fwd_n16384_d128",
+         "bwd_ext_n4096_d128", "fwd_bias_n4096_d128", "bwd_bias_n4096_d128", "fwd_drop_n4096_d128",
+         "bwd_drop_n4096_d128", "decode", "fwd_long", "bwd_long", "bwd_n16384_d128", "fwd_n16384_d128",
          "bwd_n4096_d64", "fwd_n4096_d64", "bwd_det_n4096_d128")
 
 
@@ -661,7 +662,7 @@ def run_case(args):
         o, lse = fa.attention_forward(q, k, v, causal=causal, scale=cfg.scale)
         ff = W.flops_forward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal)
         fb = W.flops_backward(cfg.B, cfg.H, cfg.Nq, cfg.Nk, cfg.d, causal)
-        if name.startswith(("bwd", "fwd_ext")):
+        if name.startswith("bwd"):
             ws = torch.empty(fa.fa_bwd_workspace_size(cfg.B, cfg.H, cfg.Nq, cfg.d), dtype=torch.uint8, device=dev)
             dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
         if name.startswith("fwd_fp8"):
@@ -671,15 +672,19 @@ def run_case(args):
             v8, dsv = fa.quantize_fp8(v, None, False, stream)
             fn = lambda: fa.fa_fwd_fp8(q8, k8, v8, dsq, dsk, dsv, o, lse, causal, cfg.scale, stream)
             units = ff / 1e12
-        elif "_ext_" in name:
-            gb = torch.Generator().manual_seed(9)
-            bias = (torch.randn(1, cfg.H, cfg.Nq, cfg.Nk, generator=gb) * 0.5).to(torch.bfloat16).to(dev)
-            fa.fa_fwd_ext(q, k, v, o, lse, bias, causal, cfg.scale, 0.1, 1234, 0, stream)
+        elif "_ext_" in name or "_bias_" in name or "_drop_" in name:
+            # bias [1, H, N, N] and / or dropout p = 0.1 (ext: both)
+            bias = None
+            if "_drop_" not in name:
+                gb = torch.Generator().manual_seed(9)
+                bias = (torch.randn(1, cfg.H, cfg.Nq, cfg.Nk, generator=gb) * 0.5).to(torch.bfloat16).to(dev)
+            pd = 0.0 if "_bias_" in name else 0.1
+            fa.fa_fwd_ext(q, k, v, o, lse, bias, causal, cfg.scale, pd, 1234, 0, stream)
             if name.startswith("fwd"):
-                fn = lambda: fa.fa_fwd_ext(q, k, v, o, lse, bias, causal, cfg.scale, 0.1, 1234, 0, stream)
+                fn = lambda: fa.fa_fwd_ext(q, k, v, o, lse, bias, causal, cfg.scale, pd, 1234, 0, stream)
                 units = ff / 1e12
             else:
-                fn = lambda: fa.fa_bwd_ext(q, k, v, o, do, lse, dq, dk, dv, ws, bias, causal, cfg.scale, 0.1, 1234, 0,
+                fn = lambda: fa.fa_bwd_ext(q, k, v, o, do, lse, dq, dk, dv, ws, bias, causal, cfg.scale, pd, 1234, 0,
                                            stream)
                 units = fb / 1e12
         elif name.startswith("fwd"):

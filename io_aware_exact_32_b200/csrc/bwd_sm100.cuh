@@ -74,7 +74,8 @@ struct BwdTraits {
   static constexpr int BAR_SD_USED = BAR_S_FULL + 8;  // S^T/dP^T of block i are in registers
   static constexpr int BAR_P_FREE = BAR_S_FULL + 9;   // dV(i) has read P^T(i)
   static constexpr int BAR_DO_FREE = BAR_S_FULL + 10; // dV(i) has read dO(i) (d = 128: staging)
-  static constexpr int NBAR = BAR_DO_FREE + 1;
+  static constexpr int BAR_DQ_ISSUED = BAR_S_FULL + 11;  // issuer B has issued dQ(i): issuer A may issue dV(i)
+  static constexpr int NBAR = BAR_DQ_ISSUED + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -235,6 +236,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     mbar_init(bar(T::BAR_SD_USED), 128 * T::NCWG);
     mbar_init(bar(T::BAR_P_FREE), 1);
     mbar_init(bar(T::BAR_DO_FREE), 1);
+    mbar_init(bar(T::BAR_DQ_ISSUED), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -588,6 +590,9 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
         if (!(ok = warp_wait(bar(T::BAR_DS_READY), it & 1, abort_flag))) break;
         tc_fence_after();
         if constexpr (is_a) {
+          // dQ(i) goes to the tensor pipe first: its read-out gates the next block's dP^T, while dV(i)
+          // only has to precede the next S^T, which this issuer sends after it anyway.
+          if (DQ && !(ok = warp_wait(bar(T::BAR_DQ_ISSUED), it & 1, abort_flag))) break;
           // dV_j += P^T dO_i  (P^T from TMEM, dO MN-major).
           const uint64_t do_mn = make_sdesc_sw128(dos, T::BOX_BYTES, 1024);
 #pragma unroll
@@ -617,6 +622,8 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
               mma_ss_w(tDQ, ds_mn + (uint64_t)((kk * 2048) >> 4), k_mn + (uint64_t)((kk * 2048) >> 4), T::IDESC_DQ,
                        kk > 0 ? 1u : 0u);
             mma_commit_w(bar(T::BAR_DQ_FULL));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(T::BAR_DQ_ISSUED));
           }
           // d = 128: the next block's dP^T reuses the dQ columns, once dQ(it) is read out.
           if (!T::EARLY && more) {
