@@ -53,15 +53,17 @@ struct FwdTraits {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = 4 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
-  // barriers: q_full[2] | q_empty[2] | kv_full[NS] | kv_empty[NS] | s_full[2] | p_ready[2] | o_done[2] |
+  // barriers: q_full[2] | q_empty[2] | kv_full[NS] | kv_empty[NS] | s_full[2] | p_ready[2][2] | o_done[2] |
   //           o_free[2] | drain | merge
   static constexpr int BAR_Q_FULL = 0;
   static constexpr int BAR_Q_EMPTY = 2;
   static constexpr int BAR_KV_FULL = 4;
   static constexpr int BAR_KV_EMPTY = 4 + NS;
   static constexpr int BAR_S_FULL = 4 + 2 * NS;
+  // p_ready[t][half]: group t has written the softmax weights of keys [64 half, 64 half + 64) of
+  // its current tile (the P V product starts on the first half while the second is computed).
   static constexpr int BAR_P_READY = BAR_S_FULL + 2;
-  static constexpr int BAR_O_DONE = BAR_P_READY + 2;
+  static constexpr int BAR_O_DONE = BAR_P_READY + 4;
   static constexpr int BAR_O_FREE = BAR_O_DONE + 2;  // group t has read O_t out: the next item may overwrite it
   static constexpr int BAR_DRAIN = BAR_O_FREE + 2;
   static constexpr int BAR_MERGE = BAR_DRAIN + 1;  // split mode: group 1's row statistics published
@@ -133,12 +135,17 @@ __device__ __forceinline__ void fwd_issue_qk(uint32_t tmem_d, uint32_t q_smem, u
   }
 }
 
+// O += P V over keys [64 half, 64 half + 64) of the tile (accumulate: whether O already holds a sum;
+// the second half always accumulates).
 template <int D, bool F8>
-__device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
+__device__ __forceinline__ void fwd_issue_pv(uint32_t tmem_d, uint32_t tmem_p, uint32_t v_smem, int half,
+                                             bool accumulate) {
   using T = FwdTraits<D, F8>;
   const uint64_t vd = make_sdesc_sw128(v_smem, T::BOX_BYTES, 1024);
+  accumulate = accumulate || half > 0;
+  constexpr int NK = 128 / T::KSTEP;
 #pragma unroll
-  for (int kk = 0; kk < 128 / T::KSTEP; ++kk) {
+  for (int kk = half * NK / 2; kk < (half + 1) * NK / 2; ++kk) {
     // KSTEP keys per step: P advances 8 32-bit columns (two bf16 or four E4M3 per column), V rows
     // by KSTEP x 128 bytes.
     const uint64_t voff = (uint64_t)((kk * T::KSTEP * 128) >> 4);
@@ -250,7 +257,8 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(T::BAR_S_FULL + t), 1);
-      mbar_init(bar(T::BAR_P_READY + t), 128);
+      mbar_init(bar(T::BAR_P_READY + 2 * t), 128);
+      mbar_init(bar(T::BAR_P_READY + 2 * t + 1), 128);
       mbar_init(bar(T::BAR_O_DONE + t), 1);
       mbar_init(bar(T::BAR_O_FREE + t), 128);
     }
@@ -342,9 +350,29 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
         }
         const float base = (m_run == -INFINITY) ? 0.f : m_run;
         const float2 nb2 = make_float2(-base, -base);
-        // Exponentials in four chunks of 16 pairs; each chunk of P (bf16 pairs) is stored to TMEM
-        // as soon as it is ready.  Two row sums: exact (for LSE) and of the rounded weights
-        // (normalises O so it stays a convex combination of V rows).
+        // O_t still holds the sum through this group's previous tile: when the max moved, it is
+        // scaled before the first key half of this tile is published (after that half's weights,
+        // when the first 64 scores are no longer needed).  That P V has completed already (it was
+        // issued before this tile's S, whose completion this group has seen); the wait confirms it.
+        const bool any_resc = __any_sync(0xffffffffu, resc);
+        auto rescale_o = [&]() -> bool {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (cnt + step - 1) & 1, abort_flag)))
+            return false;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld32x32b_x16_wait(lane_addr + colO + 16 * c, o);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32x32b_x16(lane_addr + colO + 16 * c, o);
+          }
+          return true;
+        };
+        // Exponentials in four chunks of 32 keys; each chunk of P is stored to TMEM as soon as it is
+        // ready, and each key half (two chunks) is published on its own barrier so that its P V
+        // starts while the next half is computed.  Two row sums: exact (for LSE) and of the rounded
+        // weights (normalises O so it stays a convex combination of V rows).
         float2 sum_e[2], sum_r[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) sum_e[i] = sum_r[i] = make_float2(0.f, 0.f);
@@ -368,6 +396,12 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
               sum_r[1] = fadd2(sum_r[1], e4m3x2_to_f32x2(hi));
             }
             tmem_st32x32b_x8(lane_addr + colS + 8 * ch, pk);
+            if (ch == 1 && any_resc && !(ok = rescale_o())) break;
+            if (ch & 1) {
+              tmem_st_wait();
+              tc_fence_before();
+              mbar_arrive(bar(T::BAR_P_READY + 2 * t + (ch >> 1)));
+            }
           }
         } else {
 #pragma unroll
@@ -392,30 +426,19 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
               }
             }
             tmem_st32x32b_x16(lane_addr + colS + 16 * ch, pk);
+            if (ch == 1 && any_resc && !(ok = rescale_o())) break;
+            if (ch & 1) {
+              tmem_st_wait();
+              tc_fence_before();
+              mbar_arrive(bar(T::BAR_P_READY + 2 * t + (ch >> 1)));
+            }
           }
         }
+        if (!ok) break;
         const float2 tot_e = fadd2(sum_e[0], sum_e[1]);
         const float2 tot_r = fadd2(sum_r[0], sum_r[1]);
         l_run = l_run * alpha + (tot_e.x + tot_e.y);
         lr_run = lr_run * alpha + (tot_r.x + tot_r.y);
-        if (__any_sync(0xffffffffu, resc)) {
-          // O_t still holds the sum through this group's previous tile: wait until that PV has
-          // landed, then scale.
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_O_DONE + t), (cnt + step - 1) & 1, abort_flag));
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32x32b_x32_wait(lane_addr + colO + 32 * c, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32x32b_x32(lane_addr + colO + 32 * c, o);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(T::BAR_P_READY + t));
       }
       if (!ok) break;
       // This group's accumulator is complete once its last PV has landed.
@@ -502,6 +525,17 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
       };
       const uint32_t tS[2] = {tmem_base + T::col_s(0), tmem_base + T::col_s(1)};
       const uint32_t tO[2] = {tmem_base + T::col_o(0), tmem_base + T::col_o(1)};
+      // O_t += P_t V (V of load v_load): the first key half as soon as group t has published it, then
+      // the second; c counts group t's tiles (barrier phase), acc: whether O_t already holds a sum.
+      auto pv = [&](int t, int c, int v_load, bool acc) -> bool {
+        for (int half = 0; half < 2; ++half) {
+          if (!warp_wait(bar(T::BAR_P_READY + 2 * t + half), c & 1, abort_flag)) return false;
+          tc_fence_after();
+          fwd_issue_pv<D, F8>(tO[t], tS[t], kv_smem(v_load), half, acc);
+        }
+        mma_commit_w(bar(T::BAR_O_DONE + t));
+        return true;
+      };
       bool ok = true;
       int L = 0;                // global index of the item's first K/V load
       int cnt0 = 0, cnt1 = 0;   // S tiles of groups 0 / 1 in earlier items (barrier phases run on)
@@ -533,10 +567,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
             release(ik0);
             if (v1_prev >= 0) {
               if (!(ok = kv_wait(v1_prev))) break;
-              if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (cnt1 + i - 1) & 1, abort_flag))) break;
-              tc_fence_after();
-              fwd_issue_pv<D, F8>(tO[1], tS[1], kv_smem(v1_prev), i - 1 > 0);
-              mma_commit_w(bar(T::BAR_O_DONE + 1));
+              if (!(ok = pv(1, cnt1 + i - 1, v1_prev, i - 1 > 0))) break;
               release(v1_prev);
               v1_prev = -1;
             }
@@ -549,20 +580,12 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
               v1_prev = iv1;
             }
             if (!(ok = kv_wait(iv0))) break;
-            if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), (cnt0 + i) & 1, abort_flag))) break;
-            tc_fence_after();
-            fwd_issue_pv<D, F8>(tO[0], tS[0], kv_smem(iv0), i > 0);
-            mma_commit_w(bar(T::BAR_O_DONE + 0));
+            if (!(ok = pv(0, cnt0 + i, iv0, i > 0))) break;
             release(iv0);
           }
           if (ok && v1_prev >= 0) {
             const int i = nsteps - 1;
-            if ((ok = kv_wait(v1_prev)) && (ok = warp_wait(bar(T::BAR_P_READY + 1), (cnt1 + i) & 1, abort_flag))) {
-              tc_fence_after();
-              fwd_issue_pv<D, F8>(tO[1], tS[1], kv_smem(v1_prev), i > 0);
-              mma_commit_w(bar(T::BAR_O_DONE + 1));
-              release(v1_prev);
-            }
+            if ((ok = kv_wait(v1_prev)) && (ok = pv(1, cnt1 + i, v1_prev, i > 0))) release(v1_prev);
           }
           cnt0 += (n_kv + 1) / 2;
           cnt1 += n_kv / 2;
@@ -580,10 +603,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
             }
             if (j > 0) {
               if (j == 1 && !(ok = o_free(1))) break;
-              if (!(ok = warp_wait(bar(T::BAR_P_READY + 1), (cnt1 + j - 1) & 1, abort_flag))) break;
-              tc_fence_after();
-              fwd_issue_pv<D, F8>(tO[1], tS[1], kv_smem(v_prev), j - 1 > 0);
-              mma_commit_w(bar(T::BAR_O_DONE + 1));
+              if (!(ok = pv(1, cnt1 + j - 1, v_prev, j - 1 > 0))) break;
               release(v_prev);
             }
             fwd_issue_qk<D, F8>(tS[1], q_smem[1], kv_smem(ik));
@@ -592,20 +612,12 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
             if (!(ok = kv_wait(iv))) break;
             if (j < w.n0) {
               if (j == 0 && !(ok = o_free(0))) break;
-              if (!(ok = warp_wait(bar(T::BAR_P_READY + 0), (cnt0 + j) & 1, abort_flag))) break;
-              tc_fence_after();
-              fwd_issue_pv<D, F8>(tO[0], tS[0], kv_smem(iv), j > 0);
-              mma_commit_w(bar(T::BAR_O_DONE + 0));
+              if (!(ok = pv(0, cnt0 + j, iv, j > 0))) break;
             }
             v_prev = iv;
           }
           if (ok && w.n_kv == 1) ok = o_free(1);
-          if (ok && (ok = warp_wait(bar(T::BAR_P_READY + 1), (cnt1 + w.n_kv - 1) & 1, abort_flag))) {
-            tc_fence_after();
-            fwd_issue_pv<D, F8>(tO[1], tS[1], kv_smem(v_prev), w.n_kv - 1 > 0);
-            mma_commit_w(bar(T::BAR_O_DONE + 1));
-            release(v_prev);
-          }
+          if (ok && (ok = pv(1, cnt1 + w.n_kv - 1, v_prev, w.n_kv - 1 > 0))) release(v_prev);
           cnt0 += w.n0;
           cnt1 += w.n1;
         }
