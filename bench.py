@@ -623,7 +623,7 @@ def small_step(fa, W, dev, stream, peaks, flush_buf, reps=200):
 CASES = ("fwd_c2", "bwd_c2", "fwd_n4096_d128", "bwd_n4096_d128", "fwd_fp8_n4096_d128", "fwd_ext_n4096_d128",
          "bwd_ext_n4096_d128", "fwd_bias_n4096_d128", "bwd_bias_n4096_d128", "fwd_drop_n4096_d128",
          "bwd_drop_n4096_d128", "decode", "fwd_long", "bwd_long", "bwd_n16384_d128", "fwd_n16384_d128",
-         "bwd_n4096_d64", "fwd_n4096_d64", "bwd_det_n4096_d128")
+         "bwd_n4096_d64", "fwd_n4096_d64", "bwd_det_n4096_d128", "quant_n4096_d128")
 
 
 def run_case(args):
@@ -665,7 +665,21 @@ def run_case(args):
         if name.startswith("bwd"):
             ws = torch.empty(fa.fa_bwd_workspace_size(cfg.B, cfg.H, cfg.Nq, cfg.d), dtype=torch.uint8, device=dev)
             dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-        if name.startswith("fwd_fp8"):
+        if name.startswith("quant"):
+            # Q and K rotated (random-sign Hadamard) and quantised, V quantised; algorithmic bytes: read
+            # bf16 and write E4M3 once (3 bytes an element).
+            signs = W.make_hadamard_signs(cfg.d, 11).to(dev)
+            q8, dsq = fa.quantize_fp8(q, signs, True, stream)
+            k8, dsk = fa.quantize_fp8(k, signs, True, stream)
+            v8, dsv = fa.quantize_fp8(v, None, False, stream)
+
+            def fn():
+                fa.fa_quantize_fp8(q, signs, q8, dsq, True, stream)
+                fa.fa_quantize_fp8(k, signs, k8, dsk, True, stream)
+                fa.fa_quantize_fp8(v, None, v8, dsv, False, stream)
+
+            units, unit = 3 * q.numel() * 3 / 1e9, "GB/s"
+        elif name.startswith("fwd_fp8"):
             signs = W.make_hadamard_signs(cfg.d, 11).to(dev)
             q8, dsq = fa.quantize_fp8(q, signs, True, stream)
             k8, dsk = fa.quantize_fp8(k, signs, True, stream)
@@ -694,7 +708,8 @@ def run_case(args):
             det = name.startswith("bwd_det")
             fn = lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, causal, cfg.scale, stream, deterministic=det)
             units = fb / 1e12
-        unit = "TFLOP/s"
+        if not name.startswith("quant"):
+            unit = "TFLOP/s"
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         fn()

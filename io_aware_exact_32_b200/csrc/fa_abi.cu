@@ -420,7 +420,8 @@ fa_status fa_quantize_fp8(const void* x, const float* signs, void* x8, float* de
   // The descale buffer first holds the per-head amax (float bits, atomically maximised).
   if (cudaMemsetAsync(descale, 0, (size_t)BH * sizeof(float), s) != cudaSuccess) return FA_ERR_CUDA;
   if (N > 0) {
-    const int chunks = (N + fa::kQuantRowsPerBlock - 1) / fa::kQuantRowsPerBlock;
+    const int rows = d == 64 ? fa::kQuantRows<64> : fa::kQuantRows<128>;
+    const int chunks = (N + rows - 1) / rows;
     const long long blocks = BH * chunks;
     if (blocks > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
     const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
