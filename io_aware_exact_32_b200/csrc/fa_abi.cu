@@ -70,8 +70,9 @@ bool make_map_3d_f32(CUtensorMap* map, void* base, int D, int N, long long BH) {
   return r == CUDA_SUCCESS;
 }
 
-// [planes, Nq, Nk] bf16 bias viewed as {Nk, Nq, planes}; box = 64 keys x 128 query rows x 1, used only
-// for L2 prefetches.  Rows past Nq and keys past Nk are clipped.
+// [planes, Nq, Nk] bf16 bias viewed as {Nk, Nq, planes}; box = 64 keys x 128 query rows x 1, 128-byte
+// swizzle: the forward stages bias tiles through it, the backward prefetches them into L2.  Rows past
+// Nq and keys past Nk read as zero.
 bool make_map_bias(CUtensorMap* map, const void* base, int Nk, int Nq, long long planes) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
@@ -199,7 +200,7 @@ fa_status launch_fwd(const void* q, const void* k, const void* v, void* o, float
                      float scale, int causal, cudaStream_t stream, const float* descale_q = nullptr,
                      const float* descale_k = nullptr, const float* descale_v = nullptr,
                      const ExtArgs* ext = nullptr) {
-  using T = fa::FwdTraits<D, F8>;
+  using T = fa::FwdTraits<D, F8, EXT>;
   CUtensorMap mq, mk, mv;
   if (!make_map_3d(&mq, q, D, Nq, BH, F8) || !make_map_3d(&mk, k, D, Nk, BH, F8) ||
       !make_map_3d(&mv, v, D, Nk, BH, F8))

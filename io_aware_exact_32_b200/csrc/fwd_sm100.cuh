@@ -35,7 +35,7 @@ namespace fa {
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, bool EXT = false>
 struct FwdTraits {
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(!F8 || D == 128, "FP8 operands: d = 128");
@@ -48,13 +48,18 @@ struct FwdTraits {
   static constexpr int TILE_BYTES = NBOX * BOX_BYTES;  // one 128 x D tile
   static constexpr int KSTEP = 32 / EB;                // MMA K per instruction (32 bytes of operand)
   static constexpr int NS = F8 ? 8 : ((D == 64) ? 6 : 3);  // K/V ring stages
-  // Two Q slots (work items alternate between them, so the next item's Q loads while the current
-  // one runs), each holding the item's two 128-row tiles: slot s, tile t at OFF_Q + (2 s + t) TILE_BYTES.
+  // Q slots (work items alternate between them, so the next item's Q loads while the current one
+  // runs), each holding the item's two 128-row tiles: slot s, tile t at OFF_Q + (2 s + t) TILE_BYTES.
+  // The bias instantiation keeps one slot and spends the space on two bias tiles (one per softmax
+  // group: 128 rows x 128 keys bf16, two 64-key TMA boxes with the 128-byte swizzle).
+  static constexpr int QSLOTS = EXT ? 1 : 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = 4 * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NS * TILE_BYTES;
+  static constexpr int OFF_KV = 2 * QSLOTS * TILE_BYTES;
+  static constexpr int BIAS_TILE = 128 * 128 * 2;
+  static constexpr int OFF_BIAS = OFF_KV + NS * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_BIAS + (EXT ? 2 * BIAS_TILE : 0);
   // barriers: q_full[2] | q_empty[2] | kv_full[NS] | kv_empty[NS] | s_full[2] | p_ready[2][2] | o_done[2] |
-  //           o_free[2] | drain | merge
+  //           o_free[2] | drain | merge | bias_full[2] | bias_empty[2]
   static constexpr int BAR_Q_FULL = 0;
   static constexpr int BAR_Q_EMPTY = 2;
   static constexpr int BAR_KV_FULL = 4;
@@ -67,14 +72,18 @@ struct FwdTraits {
   static constexpr int BAR_O_FREE = BAR_O_DONE + 2;  // group t has read O_t out: the next item may overwrite it
   static constexpr int BAR_DRAIN = BAR_O_FREE + 2;
   static constexpr int BAR_MERGE = BAR_DRAIN + 1;  // split mode: group 1's row statistics published
-  static constexpr int NBAR = BAR_MERGE + 1;
+  static constexpr int BAR_BIAS_FULL = BAR_MERGE + 1;       // group t's bias tile has landed
+  static constexpr int BAR_BIAS_EMPTY = BAR_BIAS_FULL + 2;  // group t has read its bias tile
+  static constexpr int NBAR = BAR_BIAS_EMPTY + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // tmem base (u32), abort flag (int)
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
   // TMEM columns: S_t at 128 t, O_t at 256 + D t.
   static __host__ __device__ constexpr uint32_t col_s(int t) { return 128u * t; }
   static __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + (uint32_t)D * t; }
-  static constexpr int THREADS = 320;  // warps 0-7 softmax, 8 MMA issuer, 9 TMA
+  // Warps 0-7 softmax, 8 MMA issuer, 9 TMA (Q, K, V), 10 (bias instantiation) TMA of the bias tiles.
+  static constexpr int WARP_BIAS = 10;
+  static constexpr int THREADS = EXT ? 352 : 320;
   static constexpr uint32_t IDESC_QK = F8 ? make_idesc_e4m3(128, 128, false, false) : make_idesc_bf16(128, 128, false, false);
   static constexpr uint32_t IDESC_PV = F8 ? make_idesc_e4m3(128, D, false, true) : make_idesc_bf16(128, D, false, true);
 };
@@ -178,21 +187,15 @@ __device__ __forceinline__ float max64(const float* s) {
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-// Bias step of the EXT forward for 64 keys [k0, k0 + 64) of one row: s <- s * scale_log2 + bias * log2(e)
-// (a key past Nk reads no bias; it is already -inf).  Rows are read as 16-byte chunks, so Nk is a
-// multiple of 8 whenever a bias is given.
-__device__ __forceinline__ void fwd_apply_bias(float* s, const __nv_bfloat16* bias_row, int k0, int Nk,
-                                               float scale_log2) {
+// Bias step of the EXT forward for the 64 keys of one row held in a staged bias box:
+// s <- s * scale_log2 + bias * log2(e).  The box is 128 rows of 128 bytes with 16-byte chunk c of row
+// r at ((c ^ (r % 8)) * 16) (the 128-byte swizzle of the TMA box); keys past Nk and rows past Nq
+// were filled with zeros by the TMA (those scores are -inf or never stored).
+__device__ __forceinline__ void fwd_apply_bias_smem(float* s, const uint8_t* box, int r, float scale_log2) {
   constexpr float kLog2eF = 1.4426950408889634f;
-  if (bias_row == nullptr) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c) s[c] *= scale_log2;
-    return;
-  }
 #pragma unroll
   for (int g = 0; g < 8; ++g) {
-    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
-    if (k0 + 8 * g < Nk) raw = __ldg(reinterpret_cast<const uint4*>(bias_row + k0 + 8 * g));
+    const uint4 raw = *reinterpret_cast<const uint4*>(box + r * 128 + ((g ^ (r & 7)) << 4));
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -204,12 +207,12 @@ __device__ __forceinline__ void fwd_apply_bias(float* s, const __nv_bfloat16* bi
 
 // EXT: the scores get an additive bias (p.bias) and the weights dropout (p.drop) before P V.
 template <int D, bool F8 = false, bool EXT = false>
-__global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
+__global__ void __launch_bounds__(FwdTraits<D, F8, EXT>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmB,
                   const FwdParams p) {
   static_assert(!(F8 && EXT), "bias and dropout are not combined with FP8 operands");
-  using T = FwdTraits<D, F8>;
+  using T = FwdTraits<D, F8, EXT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -245,6 +248,11 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
   }
   int issued = 0;           // K/V loads started by the TMA producer (its lane 0), for the teardown
   int q_fills[2] = {0, 0};  // Q loads per slot started by the TMA producer, for the teardown
+  int b_fills[2] = {0, 0};  // bias tiles per group started by the bias loader, for the teardown
+  const bool staged_bias = EXT && p.bias != nullptr;
+  // Bias tiles group t consumes in item w, in its order: its key tiles j (two tiles: 0 .. n_t - 1;
+  // split: t, t + 2, ...).
+  auto n_bias = [&](const FwdItem& w, int t) { return two ? (t ? w.n1 : w.n0) : (w.n_kv + 1 - t) / 2; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -264,6 +272,10 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
     }
     mbar_init(bar(T::BAR_DRAIN), 1);
     mbar_init(bar(T::BAR_MERGE), 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(T::BAR_BIAS_FULL + t), 1);
+      mbar_init(bar(T::BAR_BIAS_EMPTY + t), 128);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -275,8 +287,8 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    if (EXT && p.bias != nullptr) tma_prefetch_desc(&tmB);
   }
+  if (warp == T::WARP_BIAS && lane == 0 && staged_bias) tma_prefetch_desc(&tmB);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -292,7 +304,8 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
     const uint32_t colS = T::col_s(t), colO = T::col_o(t);
     bool ok = true;
-    int cnt = 0;  // S tiles this group has processed in earlier items (barrier phases run on)
+    int cnt = 0;   // S tiles this group has processed in earlier items (barrier phases run on)
+    int bcnt = 0;  // staged bias tiles this group has consumed
     for (int it = 0; ok && item_at(it) < n_items; ++it) {
       const FwdItem w = decode(item_at(it));
       const int bh = w.bh;
@@ -306,11 +319,8 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
       // EXT: the scores are turned into log2-domain logits s * scale * log2(e) + bias * log2(e) in
       // place, so the exponent step below multiplies by 1.
       const float2 sc2 = EXT ? make_float2(1.f, 1.f) : make_float2(scale_log2, scale_log2);
-      const __nv_bfloat16* bias_row = nullptr;
-      if constexpr (EXT) {
-        if (p.bias != nullptr && row < p.Nq)
-          bias_row = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + (size_t)row * p.Nk;
-      }
+      // EXT with a bias: this group's staged bias tile, one 64-key box per half of the scores.
+      const uint8_t* bias_box = smem + T::OFF_BIAS + t * T::BIAS_TILE;
       for (int step = 0; step < n_own; ++step) {
         const int j = two ? step : 2 * step + t;  // key tile
         ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL + t), (cnt + step) & 1, abort_flag));
@@ -330,7 +340,16 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
           for (int c = 0; c < 64; ++c)
             if (c > lim) s[c] = -INFINITY;
         }
-        if constexpr (EXT) fwd_apply_bias(s, bias_row, 128 * j, p.Nk, scale_log2);
+        if constexpr (EXT) {
+          if (staged_bias) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_BIAS_FULL + t), bcnt & 1, abort_flag));
+            if (!ok) break;
+            fwd_apply_bias_smem(s, bias_box, r, scale_log2);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s[c] *= scale_log2;
+          }
+        }
         const float mx_a = max64(s);
         tmem_wait_ld_x64(sb);
         if (masked) {
@@ -338,7 +357,16 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
           for (int c = 0; c < 64; ++c)
             if (c + 64 > lim) s2[c] = -INFINITY;
         }
-        if constexpr (EXT) fwd_apply_bias(s2, bias_row, 128 * j + 64, p.Nk, scale_log2);
+        if constexpr (EXT) {
+          if (staged_bias) {
+            fwd_apply_bias_smem(s2, bias_box + T::BIAS_TILE / 2, r, scale_log2);
+            mbar_arrive(bar(T::BAR_BIAS_EMPTY + t));  // this tile's bias has been read
+            ++bcnt;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) s2[c] *= scale_log2;
+          }
+        }
         const float mx = fmaxf(mx_a, max64(s2));
         const float m_tile = EXT ? mx : mx * scale_log2;
         float alpha = 1.f;
@@ -541,10 +569,10 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
       int cnt0 = 0, cnt1 = 0;   // S tiles of groups 0 / 1 in earlier items (barrier phases run on)
       for (int k = 0; ok && item_at(k) < n_items; ++k) {
         const FwdItem w = decode(item_at(k));
-        const int slot = k & 1;
+        const int slot = k % T::QSLOTS;
         const uint32_t q_smem[2] = {sbase + T::OFF_Q + (2 * slot) * T::TILE_BYTES,
                                     sbase + T::OFF_Q + (2 * slot + 1) * T::TILE_BYTES};
-        if (!(ok = warp_wait(bar(T::BAR_Q_FULL + slot), (k >> 1) & 1, abort_flag))) break;
+        if (!(ok = warp_wait(bar(T::BAR_Q_FULL + slot), (k / T::QSLOTS) & 1, abort_flag))) break;
         // The first P V of group t in this item overwrites O_t: group t must have read out the
         // previous item's output (two-tile mode; the split mode has one item per CTA).
         auto o_free = [&](int t) {
@@ -623,22 +651,24 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
         }
         // Every S MMA of this item has been issued: its Q slot is free once they complete (the
         // commit tracks all earlier MMAs of this thread).  Only slots the producer refills.
-        if (ok && k + 2 < my_items) mma_commit_w(bar(T::BAR_Q_EMPTY + slot));
+        if (ok && k + T::QSLOTS < my_items) mma_commit_w(bar(T::BAR_Q_EMPTY + slot));
         L += 2 * w.n_kv;
       }
       if (!ok) *abort_flag = 1;
     }
     __syncwarp();
-  } else {
+  } else if (warp == 9) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       bool ok = true;
       int L = 0;  // global index of the item's first K/V load
       for (int k = 0; ok && item_at(k) < n_items; ++k) {
         const FwdItem w = decode(item_at(k));
-        const int slot = k & 1;
-        // The slot's previous item (k - 2) must have finished its S MMAs.
-        if (k >= 2 && !(ok = mbar_wait(bar(T::BAR_Q_EMPTY + slot), ((k - 2) >> 1) & 1, abort_flag))) break;
+        const int slot = k % T::QSLOTS;
+        // The slot's previous item (k - QSLOTS) must have finished its S MMAs.
+        if (k >= T::QSLOTS &&
+            !(ok = mbar_wait(bar(T::BAR_Q_EMPTY + slot), ((k - T::QSLOTS) / T::QSLOTS) & 1, abort_flag)))
+          break;
         mbar_arrive_expect_tx(bar(T::BAR_Q_FULL + slot), p.tiles * T::TILE_BYTES);
         for (int t = 0; t < p.tiles; ++t)
           for (int b = 0; b < T::NBOX; ++b)
@@ -655,17 +685,38 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
             tma_load_3d(sbase + T::OFF_KV + s * T::TILE_BYTES + b * T::BOX_BYTES, map, bar(T::BAR_KV_FULL + s),
                         T::BOX_COLS * b, 128 * (idx >> 1), w.bh);
           issued = g + 1;
-          if constexpr (EXT) {
-            // Warm the L2 with the bias tiles of this key tile (each softmax row reads its 256 bytes
-            // with plain loads about NS loads later).
-            if (p.bias != nullptr && !(idx & 1)) {
-              const int plane = (w.bh / p.H) * p.bias_pb + (w.bh % p.H) * p.bias_ph;
-              for (int t = 0; t < p.tiles; ++t)
-                for (int b = 0; b < 2; ++b) tma_prefetch_l2_3d(&tmB, 128 * (idx >> 1) + 64 * b, w.q0 + 128 * t, plane);
-            }
-          }
         }
         L += 2 * w.n_kv;
+      }
+      if (!ok) *abort_flag = 1;
+    }
+    __syncwarp();
+  } else if (EXT && warp == T::WARP_BIAS) {
+    // ------------------------------------------------------------------ bias tiles (TMA)
+    // Group t's next bias tile goes into its buffer as soon as the group has read the previous one;
+    // the tiles follow each group's own order of key tiles, the two groups interleaved.  A group
+    // releases a tile using only tiles loaded before it, so the interleaving cannot deadlock.
+    if (lane == 0 && staged_bias) {
+      bool ok = true;
+      for (int k = 0; ok && item_at(k) < n_items; ++k) {
+        const FwdItem w = decode(item_at(k));
+        const int plane = (w.bh / p.H) * p.bias_pb + (w.bh % p.H) * p.bias_ph;
+        const int nb0 = n_bias(w, 0), nb1 = n_bias(w, 1);
+        for (int st = 0; ok && st < max(nb0, nb1); ++st) {
+          for (int t = 0; t < 2; ++t) {
+            if (st >= (t ? nb1 : nb0)) continue;
+            const int j = two ? st : 2 * st + t;  // key tile
+            const int row0 = w.q0 + (two ? 128 * t : 0);
+            if (b_fills[t] > 0 &&
+                !(ok = mbar_wait(bar(T::BAR_BIAS_EMPTY + t), (b_fills[t] - 1) & 1, abort_flag)))
+              break;
+            mbar_arrive_expect_tx(bar(T::BAR_BIAS_FULL + t), T::BIAS_TILE);
+            for (int b = 0; b < 2; ++b)
+              tma_load_3d(sbase + T::OFF_BIAS + t * T::BIAS_TILE + b * (T::BIAS_TILE / 2), &tmB,
+                          bar(T::BAR_BIAS_FULL + t), 128 * j + 64 * b, row0, plane);
+            ++b_fills[t];
+          }
+        }
       }
       if (!ok) *abort_flag = 1;
     }
@@ -692,6 +743,9 @@ __global__ void __launch_bounds__(FwdTraits<D, F8>::THREADS, 1)
       drain_wait(bar(T::BAR_KV_FULL + idx % T::NS), (idx / T::NS) & 1);
     for (int slot = 0; slot < 2; ++slot)
       if (q_fills[slot] > 0) drain_wait(bar(T::BAR_Q_FULL + slot), (q_fills[slot] - 1) & 1);
+  } else if (EXT && warp == T::WARP_BIAS && lane == 0 && aborted) {
+    for (int t = 0; t < 2; ++t)
+      if (b_fills[t] > 0) drain_wait(bar(T::BAR_BIAS_FULL + t), (b_fills[t] - 1) & 1);
   }
 }
 
