@@ -553,6 +553,14 @@ def extra_measurements(fa, W, dev, stream, peaks, iters=10):
                 "fwd_bwd_tflops": (ff + fb) / (t_fe + t_be) / 1e12, "fwd_ms": 1e3 * t_fe, "bwd_ms": 1e3 * t_be,
                 "vs_plain_fwd": t_f / t_fe, "vs_plain_bwd": t_b / t_be,
                 "note": "bias [1, H, N, N] bf16, dropout p = 0.1"}
+            # Each extension alone: the bias without dropout, and dropout 0.1 without a bias.
+            for name, bias_, p_ in (("bias_only", bias, 0.0), ("dropout_only", None, 0.1)):
+                t_f1 = timed(lambda: fa.fa_fwd_ext(q, k, v, oe, lsee, bias_, True, cfg.scale, p_, 1234, 0, stream))
+                t_b1 = timed(lambda: fa.fa_bwd_ext(q, k, v, oe, do, lsee, dq, dk, dv, ws, bias_, True, cfg.scale, p_,
+                                                   1234, 0, stream))
+                res[f"{name}_causal_n4096_d128"] = {
+                    "fwd_tflops": ff / t_f1 / 1e12, "bwd_tflops": fb / t_b1 / 1e12, "fwd_ms": 1e3 * t_f1,
+                    "bwd_ms": 1e3 * t_b1, "vs_plain_fwd": t_f / t_f1, "vs_plain_bwd": t_b / t_b1}
             del bias, oe, lsee
             t_bd = timed(lambda: fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, True, cfg.scale, stream,
                                            deterministic=True))

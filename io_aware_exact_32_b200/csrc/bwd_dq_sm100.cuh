@@ -261,8 +261,7 @@ __global__ void __launch_bounds__(DqTraits<D>::THREADS, 1)
     if (!ok) {
       *abort_flag = 1;
       mma_commit_w(bar(T::BAR_DRAIN));
-      const volatile int never = 0;
-      warp_wait(bar(T::BAR_DRAIN), 0, &never);
+      warp_drain_wait(bar(T::BAR_DRAIN), 0);
     }
     __syncwarp();
   } else {
@@ -288,10 +287,9 @@ __global__ void __launch_bounds__(DqTraits<D>::THREADS, 1)
       }
       if (!ok) {
         *abort_flag = 1;
-        const volatile int never = 0;
         for (int idx = max(0, issued - T::NS); idx < issued; ++idx)
-          mbar_wait(bar(T::BAR_KV_FULL + idx % T::NS), (idx / T::NS) & 1, &never);
-        mbar_wait(bar(T::BAR_QD), 0, &never);
+          drain_wait(bar(T::BAR_KV_FULL + idx % T::NS), (idx / T::NS) & 1);
+        drain_wait(bar(T::BAR_QD), 0);
       }
     }
     __syncwarp();

@@ -115,8 +115,7 @@ __global__ void __launch_bounds__(DecTraits<D>::THREADS) fa_decode_split_kernel(
       }
       if (!ok) {
         *abort_flag = 1;
-        const volatile int never = 0;
-        for (int i = max(0, issued - T::NS); i < issued; ++i) mbar_wait(full(i % T::NS), (i / T::NS) & 1, &never);
+        for (int i = max(0, issued - T::NS); i < issued; ++i) drain_wait(full(i % T::NS), (i / T::NS) & 1);
       }
     }
     __syncwarp();

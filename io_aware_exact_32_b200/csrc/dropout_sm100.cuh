@@ -84,15 +84,16 @@ __device__ __forceinline__ void dropout_keep_rowwise(const DropoutCfg& dc, uint3
   }
 }
 
-// Backward: the keep bytes of key row `key` (lane = key % 4 within its quad) for the 16 query
-// rows [4 I0, 4 I0 + 16): out[4 u + m] is 0xff if (query 4 (I0 + u) + m, key) is kept, else 0.
+// Backward: the keep decisions of key row `key` (lane = key % 4 within its quad) for the 16 query
+// rows [4 I0, 4 I0 + 16), as a mask: bit 4 u + m is set if (query 4 (I0 + u) + m, key) is kept.
 // All 32 lanes must call it together.
-__device__ __forceinline__ void dropout_keep_colwise(const DropoutCfg& dc, uint32_t I0, uint32_t key, uint32_t bh,
-                                                     int lane, uint32_t (&out)[16]) {
+__device__ __forceinline__ uint32_t dropout_keep_colwise(const DropoutCfg& dc, uint32_t I0, uint32_t key, uint32_t bh,
+                                                         int lane) {
   const int t = lane & 3;
   const uint4 w = philox4x32_10(key >> 2, I0 + t, bh, dc.offset, dc.seed_lo, dc.seed_hi);
   const uint32_t thr = dc.p8 * 0x01010101u;
   const int sh = 8 * t;
+  uint32_t mask = 0u;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int owner = (lane & ~3) | u;  // the lane that computed query quad I0 + u
@@ -100,15 +101,15 @@ __device__ __forceinline__ void dropout_keep_colwise(const DropoutCfg& dc, uint3
     const uint32_t w1 = __shfl_sync(0xffffffffu, w.y, owner);
     const uint32_t w2 = __shfl_sync(0xffffffffu, w.z, owner);
     const uint32_t w3 = __shfl_sync(0xffffffffu, w.w, owner);
-    // Byte t of each word -> one word of four bytes (query m in byte m), then compare.
+    // Byte t of each word -> one word of four bytes (query m in byte m), then compare: byte m of k
+    // is 0xff where kept; its top bit (bit 8 m + 7) goes to bit 4 u + m of the mask.
     const uint32_t packed = ((w0 >> sh) & 0xffu) | (((w1 >> sh) & 0xffu) << 8) | (((w2 >> sh) & 0xffu) << 16) |
                             (((w3 >> sh) & 0xffu) << 24);
     const uint32_t k = __vcmpgeu4(packed, thr);
-    out[4 * u + 0] = k & 0xffu;
-    out[4 * u + 1] = (k >> 8) & 0xffu;
-    out[4 * u + 2] = (k >> 16) & 0xffu;
-    out[4 * u + 3] = k >> 24;
+    const uint32_t m4 = ((k >> 7) & 1u) | ((k >> 14) & 2u) | ((k >> 21) & 4u) | ((k >> 28) & 8u);
+    mask |= m4 << (4 * u);
   }
+  return mask;
 }
 
 }  // namespace fa

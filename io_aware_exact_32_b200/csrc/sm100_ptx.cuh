@@ -119,6 +119,31 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// 16-byte shared-memory store to (row ^ x), for tiles in the 128-byte-swizzle layout: row is the
+// address of a 128-byte row (1024-byte-aligned tile) with the row's swizzle key (row index mod 8)
+// already in bits 4-6, x the chunk's unswizzled byte offset in the row (16 c, c < 8).  The XOR is
+// inside the asm so that the compiler keeps one row register instead of hoisting one address per
+// chunk out of the loops.
+__device__ __forceinline__ void st_shared_v4_xor(uint32_t row, uint32_t x, uint32_t a, uint32_t b, uint32_t c,
+                                                 uint32_t d) {
+  asm volatile("{\n\t.reg .b32 t;\n\txor.b32 t, %0, %1;\n\tst.shared.v4.b32 [t], {%2, %3, %4, %5};\n\t}" ::"r"(row),
+               "r"(x), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+// Named barrier `id` over `n` threads (a multiple of 32) that also returns whether pred held in
+// every one of them.  A group of warps that decides here whether to go on leaves its loop as a
+// whole, so no warp is left waiting at a later named barrier that the others never reach.
+__device__ __forceinline__ bool bar_sync_all(uint32_t id, uint32_t n, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return out != 0;
+}
+
 // ---------------------------------------------------------------------------------------------
 // TMA
 // ---------------------------------------------------------------------------------------------

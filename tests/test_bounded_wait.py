@@ -5,10 +5,11 @@ records FA_ERR_TIMEOUT in the device status word, the other warps of the CTA
 see its abort flag and stop, and the teardown still waits (with the fixed 2 s
 limit) for the CTA's own copies and MMAs in flight before it frees its tensor
 memory and exits.  Here the test hook fa_debug_set_wait_limit lowers the
-limit to 300 ns, so the waits of a healthy causal forward run out; the test
-checks that fa_get_device_error reports the timeout, restores the limit, and
-checks that the next forward on the same device matches the float64 oracle
-(nothing was left allocated or half-written that it could trip over).
+limit to 300 ns, so the waits of a healthy causal forward (or backward) run
+out; the test checks that fa_get_device_error reports the timeout, restores
+the limit, and checks that the next call on the same device matches the
+float64 oracle (nothing was left allocated or half-written that it could trip
+over).
 """
 import math
 
@@ -20,7 +21,7 @@ import io_aware_exact_32_b200 as fa
 from io_aware_exact_32_b200 import workloads as W
 from oracle import attention as A
 import gpu_common as gc
-from tolerances import check_lse, check_o
+from tolerances import check_grad, check_lse, check_o
 
 pytestmark = pytest.mark.gpu
 
@@ -55,3 +56,32 @@ def test_waits_give_up_and_the_device_stays_usable():
         check_o(gc.f64(o2[0, h, rows]), ro, f"O[{h}]")
         check_lse(gc.f64(lse2[0, h, rows]), rl, f"LSE[{h}]")
     assert np.isfinite(gc.f64(o2)).all()
+
+
+def test_backward_waits_give_up_and_the_device_stays_usable():
+    B, H, N, d = 1, 16, 4096, 128
+    x = W.make_attention_inputs(B, H, N, N, d, seed=92, with_do=True)
+    q, k, v, do = gc.to_dev(x["q"], x["k"], x["v"], x["do"])
+    scale = 1.0 / math.sqrt(d)
+    o, lse = fa.attention_forward(q, k, v, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    fa.fa_debug_set_wait_limit(300)
+    try:
+        fa.attention_backward(q, k, v, o, lse, do, causal=True, scale=scale)
+        torch.cuda.synchronize()
+        status = fa.fa_get_device_error()
+    finally:
+        fa.fa_debug_set_wait_limit(0)
+    assert status == FA_ERR_TIMEOUT, status
+
+    dq, dk, dv = fa.attention_backward(q, k, v, o, lse, do, causal=True, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    h = H - 1
+    _, _, rdq, rdk, rdv = A.attention_backward_full_head(gc.f64(x["q"][0, h]), gc.f64(x["k"][0, h]),
+                                                         gc.f64(x["v"][0, h]), gc.f64(x["do"][0, h]),
+                                                         scale, True, block=512, workers=4)
+    check_grad(gc.f64(dq[0, h]), rdq, "dQ")
+    check_grad(gc.f64(dk[0, h]), rdk, "dK")
+    check_grad(gc.f64(dv[0, h]), rdv, "dV")
