@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
 
   if (warp < 4 * T::NCWG) {
     // ------------------------------------------------------------------ P / dS warpgroups
-    // (d = 128: the third group is also the dQ warpgroup)
+    // (the third group is also the dQ warpgroup)
     const int wg = warp >> 2;            // which group of query columns
     const int cb = T::cb(wg);            // first query column of this group
     const int r = (warp & 3) * 32 + lane;  // key row in the block == TMEM lane (dQ: query row)
@@ -288,7 +288,6 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     constexpr bool DQ_IN_PDS = DQ;  // group 2 also reads out the dQ blocks
     const bool leader = (warp == T::WARP_DQ && lane == 0);
 
-    // P and dS of this group's query columns for block it (NCH 16-column chunks).
     // EXT: the bias entries (q, key) of one 16-column chunk of this group, as packed bf16 pairs
     // (zero past Nq or without a bias).  Loaded one chunk ahead of their use (the first chunk
     // before the block's waits), so that their latency stays off the P/dS chain.
@@ -305,6 +304,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       }
     };
 
+    // P and dS of this group's query columns for block it (NCH 16-column chunks).
     auto pds = [&](auto nch_c, int it, int q0, const uint32_t (&bias0)[8]) -> bool {
       constexpr int NCH = decltype(nch_c)::value;
       bool ok = true;
