@@ -20,13 +20,11 @@
 //         dQ block reuses the dP^T columns once dP^T has been consumed)
 //   SMEM: K_j, V_j (resident), a ring of (Q_i, dO_i) stages, dS^T (bf16, 128-byte swizzle),
 //         and at d = 64 an fp32 staging tile for the dQ block
-//   P/dS warpgroups: one thread per key row, the 128 query columns split between three groups
-//              (48, 48 and 32 columns): P, dS (the critical path); group 0 also runs the dK/dV
-//              epilogue
-//   dQ warpgroup: the third P/dS group, which turns to the block's dQ once its columns are done:
-//              one thread per query row reads it out of TMEM and the block is added into the
-//              fp32 accumulator with TMA bulk reduce-adds of a staged tile (d = 64: its own
-//              staging buffer; d = 128: the block's dO tile once dV has read it)
+//   P/dS warpgroups: one thread per key row, two groups of 64 query columns each: P, dS (the
+//              critical path); group 0 also runs the dK/dV epilogue
+//   dQ warpgroup: one thread per query row of the dQ block: read it out of TMEM, release the
+//              columns, then add it into the fp32 accumulator with TMA bulk reduce-adds of a staged
+//              tile (d = 64: its own staging buffer; d = 128: the block's dO tile once dV has read it)
 //   MMA issuer A (S^T, dV: the users of the S^T/P^T columns), MMA issuer B (dP^T, dQ, dK),
 //   and a TMA producer warp.
 // Two issuers because one thread issues at most one 128 x N x 16 MMA every ~115 cycles
@@ -83,27 +81,21 @@ struct BwdTraits {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S = 0, COL_DP = 128, COL_DV = 256, COL_DK = 256 + D;
   static constexpr uint32_t COL_DQ = SEP_DQ ? 256 + 2 * D : COL_DP;
-  // Three P/dS warpgroups split the 128 query columns of every key row, 48, 48 and 32 (the per-row
-  // chain of TMEM loads and exponentials is the critical path); the third is the dQ warpgroup,
-  // which reads out the block's dQ once its columns are done.  d = 64: P^T has its own 64 TMEM
-  // columns (bf16 pairs, the groups' parts side by side), so the next block's S^T can be computed
-  // while this block's P^T still feeds dV.  d = 128: no room; each group's P^T overwrites the
-  // start of its own, already read, columns of S^T.
+  // Two P/dS warpgroups split the 128 query columns of every key row (the per-row chain of TMEM
+  // loads and exponentials is the critical path); each writes its 64 columns of P^T (32 TMEM
+  // columns of bf16 pairs).  d = 64: P^T has its own 64 columns, so the next block's S^T can be
+  // computed while this block's P^T still feeds dV.  d = 128: no room; each group's P^T
+  // overwrites the start of its own, already read, half of S^T.
   static constexpr bool EARLY = SEP_DQ;
   static constexpr uint32_t COL_P = EARLY ? 256 + 3 * D : COL_S;
-  static constexpr int NCWG = 3;
-  static __host__ __device__ constexpr int cw(int g) { return g < 2 ? 48 : 32; }
-  static __host__ __device__ constexpr int cb(int g) { return 48 * g; }
-  // First TMEM column of group g's P^T.
-  static __host__ __device__ constexpr uint32_t p_base(int g) {
-    return EARLY ? COL_P + (uint32_t)cb(g) / 2u : COL_S + (uint32_t)cb(g);
+  static constexpr uint32_t P_WG_STRIDE = EARLY ? 32 : 64;  // TMEM columns between the groups' P^T
+  static __host__ __device__ constexpr uint32_t p_col(int kk) {  // P^T columns of K-step kk (16 queries)
+    return COL_P + (uint32_t)(kk / 4) * P_WG_STRIDE + (uint32_t)(kk % 4) * 8;
   }
-  // P^T columns of K-step kk (queries 16 kk ... 16 kk + 15, eight TMEM columns).
-  static __host__ __device__ constexpr uint32_t p_col(int kk) {
-    return p_base(16 * kk / cb(1)) + 8u * (uint32_t)(kk - cb(16 * kk / cb(1)) / 16);
-  }
-  static constexpr int WARP_DQ = 8;                     // first warp of the dQ warpgroup
-  static constexpr int WARP_A = 12, WARP_B = 13, WARP_TMA = 14;
+  static constexpr int NCWG = 2;
+  static constexpr int CW = 128 / NCWG;                 // query columns per P/dS warpgroup
+  static constexpr int WARP_DQ = 4 * NCWG;              // first warp of the dQ warpgroup
+  static constexpr int WARP_A = WARP_DQ + 4, WARP_B = WARP_DQ + 5, WARP_TMA = WARP_DQ + 6;
   static constexpr int THREADS = 32 * (WARP_TMA + 1);
   static constexpr uint32_t IDESC_SQ = make_idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
   static constexpr uint32_t IDESC_DVK = make_idesc_bf16(128, D, false, true);    // P^T dO, dS^T Q
@@ -173,9 +165,6 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __r
   reinterpret_cast<uint4*>(dq)[i] =
       make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
 }
-
-// Bits of float(bits) * s (the dQ staging stores take 32-bit words).
-__device__ __forceinline__ uint32_t scaled_bits(uint32_t bits, float s) { return __float_as_uint(__uint_as_float(bits) * s); }
 
 // First query block that sees key k0, under the bottom-right causal alignment.
 __device__ __forceinline__ int bwd_first_q_tile(int k0, int Nq, int Nk, int causal) {
@@ -268,26 +257,22 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 4 * T::NCWG) {
-    // ------------------------------------------------------------------ P / dS warpgroups
-    // (the third group is also the dQ warpgroup)
-    const int wg = warp >> 2;            // which group of query columns
-    const int cb = T::cb(wg);            // first query column of this group
-    const int r = (warp & 3) * 32 + lane;  // key row in the block == TMEM lane (dQ: query row)
+  if (warp < T::WARP_DQ) {
+    // ------------------------------------------------------------------ P / dS warpgroup(s)
+    const int wg = warp >> 2;            // which half of the query columns
+    const int cb = wg * T::CW;           // first query column of this group
+    const int r = (warp & 3) * 32 + lane;  // key row in the block == TMEM lane
     const int key = k0 + r;
     const bool key_ok = key < p.Nk;
     const uint32_t lane_addr = tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
     // Query column c of block i sees this key iff c >= cmin (bottom-right causal alignment).
     const int shift = key - (p.Nk - p.Nq);
-    const uint32_t ds_row = (sbase + T::OFF_DS + r * 128) | ((uint32_t)(r & 7) << 4);  // + swizzle key
+    const uint32_t ds_row = sbase + T::OFF_DS + r * 128;
     // EXT: this key's column of the bias (element (q, key) at bias_col[q * Nk]).
     const __nv_bfloat16* bias_col = nullptr;
     if constexpr (EXT) {
       if (p.bias != nullptr && key_ok) bias_col = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + key;
     }
-    constexpr bool DQ_IN_PDS = DQ;  // group 2 also reads out the dQ blocks
-    const bool leader = (warp == T::WARP_DQ && lane == 0);
-
     // EXT: the bias entries (q, key) of one 16-column chunk of this group, as packed bf16 pairs
     // (zero past Nq or without a bias).  Loaded one chunk ahead of their use (the first chunk
     // before the block's waits), so that their latency stays off the P/dS chain.
@@ -303,16 +288,41 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
         dst[e / 2] = lo | (hi << 16);
       }
     };
-
-    // P and dS of this group's query columns for block it (NCH 16-column chunks).
-    auto pds = [&](auto nch_c, int it, int q0, const uint32_t (&bias0)[8]) -> bool {
-      constexpr int NCH = decltype(nch_c)::value;
-      bool ok = true;
+    bool ok = true;
+    for (int it = 0; it < n_q; ++it) {
+      const int q0 = (i0 + it) * 128;
       [[maybe_unused]] uint32_t braw[2][8];
-      if constexpr (EXT) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) braw[0][i] = bias0[i];
+      if constexpr (EXT) load_bias(q0, 0, braw[0]);
+      // Per-block statistics, stored negated: -LSE in log2 units (-inf past Nq) and -D.  The
+      // first barrier keeps the previous block's readers ahead of the overwrite, the second
+      // publishes the new values.
+      {
+        const int q = q0 + r;
+        const bool in = q < p.Nq;
+        const size_t gi = (size_t)bh * p.Nq + (in ? q : 0);
+        float nlse2 = in ? -p.lse[gi] * kLog2e : -INFINITY;
+        // EXT: a row the bias hides entirely has LSE = -inf; keep its weights at 0 (a -inf bias
+        // entry plus +inf would be NaN).
+        if constexpr (EXT) nlse2 = (nlse2 == INFINITY) ? -INFINITY : nlse2;
+        const float nd = in ? -p.dvec[gi] : 0.f;
+        asm volatile("bar.sync 1, %0;" ::"n"(128 * T::NCWG) : "memory");
+        if (wg == 0) {
+          stat[r] = nlse2;
+          stat[128 + r] = nd;
+        }
       }
+      // The second barrier is also where the groups agree to go on: a wait that gave up in any of
+      // their warps ends the loop for all of them, so none is left at a later named barrier.
+      if (!bar_sync_all(1, 128 * T::NCWG, ok)) {
+        ok = false;
+        break;
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL), it & 1, abort_flag));
+      if (!ok) {
+        *abort_flag = 1;  // the other warps' waits give up at once
+        continue;         // to the agreement at the next block's barrier
+      }
+      tc_fence_after();
       const int cmin = p.causal ? shift - q0 : -1;
       // Masking is needed only where this warp holds a key past Nk or a causally hidden entry.
       const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > cb);
@@ -321,6 +331,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       [[maybe_unused]] const float zscale = p.drop.p8 != 0 ? p.drop.scale : 1.f;
       // 16-column chunks, double-buffered: the load of chunk c+1 is issued right after chunk c
       // has arrived and overlaps its arithmetic (a TMEM load wait covers every load in flight).
+      constexpr int NCH = T::CW / 16;  // 16-column chunks of this group
       uint32_t sv[2][16], dpv[2][16];
       tmem_ld32x32b_x16_nowait(lane_addr + T::COL_S + cb, sv[0]);
       tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb, dpv[0]);
@@ -401,16 +412,18 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DS_FREE), (it - 1) & 1, abort_flag));
           tc_fence_after();
         }
-        // P^T chunk -> TMEM (bf16 pairs).  d = 128: over the consumed start of this group's columns
-        // of S^T (S_FULL also covers issuer A's dV(it-1)); d = 64: into its own columns.
-        tmem_st32x32b_x8(lane_addr + T::p_base(wg) + 8 * ch, pk);
+        // P^T chunk -> TMEM (bf16 pairs).  d = 128: over the consumed first half of S^T (S_FULL
+        // also covers issuer A's dV(it-1)); d = 64: into its own columns.
+        tmem_st32x32b_x8(lane_addr + T::COL_P + wg * T::P_WG_STRIDE + 8 * ch, pk);
         // dS^T chunk (16 query columns = two 16-byte chunks) -> shared memory, K-major with
         // 128-byte swizzle (box = 64 query columns).
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
           const int kc = cb / 8 + 2 * ch + m;  // 16-byte chunk index along the 128 query columns
-          st_shared_v4_xor(ds_row + (kc >> 3) * T::BOX_BYTES, (uint32_t)(kc & 7) << 4, dk[4 * m], dk[4 * m + 1],
-                           dk[4 * m + 2], dk[4 * m + 3]);
+          const uint32_t addr = ds_row + (kc >> 3) * T::BOX_BYTES + (((kc & 7) ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk[4 * m]), "r"(dk[4 * m + 1]),
+                       "r"(dk[4 * m + 2]), "r"(dk[4 * m + 3])
+                       : "memory");
         }
         if (ch < NCH - 1) {
           tmem_wait_ld_2x16(sv[cur ^ 1], dpv[cur ^ 1]);
@@ -421,141 +434,16 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           }
         }
       }
-      return ok;
-    };
-
-    // Group 2, after its P/dS columns: the dQ block it out of TMEM, scaled, added into the fp32
-    // accumulator by TMA bulk reduce-adds of 32-column fp32 boxes staged in shared memory (rows past
-    // Nq fall outside the tensor map and are not written).
-    //   d = 64: the block has its own TMEM columns and its own staging buffer; the columns are
-    //   released as soon as they are in registers.
-    //   d = 128: the block sits in the dP^T columns, and no shared memory is left for a separate
-    //   staging buffer: the dO tile of this block's stage is free once dV(it) has read it, and takes
-    //   the block in two 64-column halves, bulk reduce-added one after the other.  Each half is read
-    //   out of TMEM just before it is staged, and the columns are released after the second read:
-    //   the next block's dP^T, which reuses them, is queued on the tensor pipe behind dV(it) and the
-    //   next S^T anyway, and holding a half in registers across the first reduce would not fit
-    //   beside the P/dS state of this group.
-    // A warp whose wait gave up (ok false on entry or here) skips the data steps but still takes
-    // every named barrier; the group decides at the first one whether the block goes on.
-    auto dq_block = [&](int it, int q0, bool ok) -> bool {
-      uint32_t va[32], vb[32];
-      // Rows of the staging boxes: row r at r * 128 bytes of each 16 KB box, 16-byte chunk c at
-      // (c ^ r % 8) * 16 (the 128-byte swizzle of the tensor map; a quarter-warp hits distinct banks).
-      auto stage = [&](uint32_t stg, const uint32_t (&v)[32], int box) {
-        const uint32_t row = (stg + box * (128 * 128) + r * 128) | ((uint32_t)(r & 7) << 4);
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4_xor(row, (uint32_t)c << 4, scaled_bits(v[4 * c], p.scale), scaled_bits(v[4 * c + 1], p.scale),
-                           scaled_bits(v[4 * c + 2], p.scale), scaled_bits(v[4 * c + 3], p.scale));
-      };
-      auto load_pair = [&](uint32_t col) {  // TMEM columns col ... col + 63 of the dQ block
-        tmem_ld32x32b_x32_nowait(lane_addr + col, va);
-        tmem_ld32x32b_x32_nowait(lane_addr + col + 32, vb);
-        tmem_wait_ld_2x32(va, vb);
-      };
-      auto reduce_pair = [&](uint32_t stg, int x0) {  // both boxes of the staging buffer at dQ column x0
-        tma_reduce_add_3d(&tmDQ, stg, x0, q0, bh);
-        tma_reduce_add_3d(&tmDQ, stg + 128 * 128, x0 + 32, q0, bh);
-        bulk_commit_group();
-      };
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DQ_FULL), it & 1, abort_flag));
-      if constexpr (T::SEP_DQ) {
-        const uint32_t stg = sbase + T::OFF_STG;
-        if (leader && it > 0) bulk_wait_group_read0();  // the previous block is read out of the buffer
-        if (!bar_sync_all(4, 128, ok)) return false;
-        tc_fence_after();
-        load_pair(T::COL_DQ);
-        tc_fence_before();
-        mbar_arrive(bar(T::BAR_DQ_FREE));
-        stage(stg, va, 0);
-        stage(stg, vb, 1);
-        fence_proxy_async_smem();
-        asm volatile("bar.sync 4, 128;" ::: "memory");
-        if (leader) reduce_pair(stg, 0);
-      } else {
-        const int s = it % T::NS;
-        const uint32_t stg = sbase + T::OFF_QD + s * 2 * T::TILE_BYTES + T::TILE_BYTES;
-        if (ok) {
-          tc_fence_after();
-          load_pair(T::COL_DQ);
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DO_FREE), it & 1, abort_flag));
-        }
-        if (ok) {
-          stage(stg, va, 0);
-          stage(stg, vb, 1);
-          fence_proxy_async_smem();
-        }
-        if (!bar_sync_all(4, 128, ok)) return false;
-        if (leader) {
-          reduce_pair(stg, 0);
-          bulk_wait_group_read0();  // the staging buffer is read out
-        }
-        asm volatile("bar.sync 4, 128;" ::: "memory");
-        load_pair(T::COL_DQ + 64);
-        tc_fence_before();
-        mbar_arrive(bar(T::BAR_DQ_FREE));
-        stage(stg, va, 0);
-        stage(stg, vb, 1);
-        fence_proxy_async_smem();
-        asm volatile("bar.sync 4, 128;" ::: "memory");
-        if (leader) {
-          reduce_pair(stg, 64);
-          bulk_wait_group_read0();
-        }
-        asm volatile("bar.sync 4, 128;" ::: "memory");
-        if (leader && it + T::NS < n_q) mbar_arrive(bar(T::BAR_QD_EMPTY + s));
+      tmem_st_wait();  // also on the give-up path: no TMEM store is left in flight at teardown
+      if (!ok) {
+        *abort_flag = 1;
+        continue;
       }
-      return true;
-    };
-
-    bool ok = true;
-    for (int it = 0; it < n_q; ++it) {
-      const int q0 = (i0 + it) * 128;
-      [[maybe_unused]] uint32_t bias0[8];
-      if constexpr (EXT) load_bias(q0, 0, bias0);
-      // Per-block statistics of this group's query columns [cb, cb + cw), stored negated: -LSE in
-      // log2 units (-inf past Nq) and -D; thread r < cw loads query column cb + r.  Each group owns
-      // its slice of the arrays, so the groups never wait on one another here: the first barrier
-      // keeps the group's readers of the previous block ahead of the overwrite, the second
-      // publishes the new values and is where the group agrees to go on (a wait that gave up in
-      // any of its warps ends the loop for all four).
-      {
-        const int q = q0 + cb + r;
-        const bool in = r < T::cw(wg) && q < p.Nq;
-        const size_t gi = (size_t)bh * p.Nq + (in ? q : 0);
-        float nlse2 = in ? -p.lse[gi] * kLog2e : -INFINITY;
-        // EXT: a row the bias hides entirely has LSE = -inf; keep its weights at 0 (a -inf bias
-        // entry plus +inf would be NaN).
-        if constexpr (EXT) nlse2 = (nlse2 == INFINITY) ? -INFINITY : nlse2;
-        const float nd = in ? -p.dvec[gi] : 0.f;
-        asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory");
-        if (r < T::cw(wg)) {
-          stat[cb + r] = nlse2;
-          stat[128 + cb + r] = nd;
-        }
-      }
-      if (!bar_sync_all(1 + wg, 128, ok)) {
-        ok = false;
-        break;
-      }
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_S_FULL), it & 1, abort_flag));
-      if (ok) {
-        tc_fence_after();
-        if (T::cw(wg) == T::cw(0)) ok = pds(std::integral_constant<int, T::cw(0) / 16>{}, it, q0, bias0);
-        else ok = pds(std::integral_constant<int, T::cw(T::NCWG - 1) / 16>{}, it, q0, bias0);
-        tmem_st_wait();  // also on the give-up path: no TMEM store is left in flight at teardown
-      }
-      if (ok) {
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(bar(T::BAR_DS_READY));
-      }
-      if (DQ_IN_PDS && wg == 2) ok = dq_block(it, q0, ok);
-      if (!ok) *abort_flag = 1;  // the other warps' waits give up at once
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(T::BAR_DS_READY));
     }
-    if (DQ_IN_PDS && leader) bulk_wait_group0();  // every reduce-add complete before the CTA exits
-    // dK, dV epilogue (group 0 owns it; at d = 64 both groups hold the same key rows).
+    // dK, dV epilogue (group 0 owns it; both groups hold the same key rows).
     if (ok && wg == 0 && n_q > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_ACC_DONE), 0, abort_flag));
     if (!ok) {
       *abort_flag = 1;
@@ -587,6 +475,115 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
         }
       }
     }
+  } else if (warp < T::WARP_DQ + 4) {
+    // ------------------------------------------------------------------ dQ warpgroup
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // query row of the dQ block == TMEM lane
+    const uint32_t lane_addr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const bool leader = (warp == T::WARP_DQ && lane == 0);
+    const uint32_t stg_row = sbase + T::OFF_STG + r * 128;
+    bool ok = true;
+    // A warp whose wait gave up skips the data steps but still takes the first named barrier of
+    // the block, where the group decides whether to go on (so that no warp is left at a barrier
+    // the others never reach).
+    for (int it = 0; it < (DQ ? n_q : 0); ++it) {
+      const int q0 = (i0 + it) * 128;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DQ_FULL), it & 1, abort_flag));
+      if constexpr (T::SEP_DQ) {
+        uint32_t v[D];
+        if (ok) {
+          tc_fence_after();
+          tmem_ld32x32b_x64_nowait(lane_addr + T::COL_DQ, v);
+          tmem_wait_ld_x64(v);
+          // The dQ columns are free as soon as they are in registers.
+          tc_fence_before();
+          mbar_arrive(bar(T::BAR_DQ_FREE));
+        }
+        // Stage the scaled block as two 32-column fp32 boxes in the 128-byte-swizzle layout (row r
+        // at r*128 bytes of each box, 16-byte chunk c at (c ^ r%8)*16: a quarter-warp hits
+        // distinct banks), then bulk reduce-add both boxes.
+        if (leader && it > 0) bulk_wait_group_read0();  // previous tile read out of the staging buffer
+        if (!bar_sync_all(2, 128, ok)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const uint32_t addr = stg_row + (c >> 3) * (128 * 128) + (((c & 7) ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "f"(__uint_as_float(v[4 * c]) * p.scale), "f"(__uint_as_float(v[4 * c + 1]) * p.scale),
+                       "f"(__uint_as_float(v[4 * c + 2]) * p.scale), "f"(__uint_as_float(v[4 * c + 3]) * p.scale)
+                       : "memory");
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        if (leader) {
+          // Rows past Nq fall outside the tensor map and are not written.
+          tma_reduce_add_3d(&tmDQ, sbase + T::OFF_STG, 0, q0, bh);
+          tma_reduce_add_3d(&tmDQ, sbase + T::OFF_STG + 128 * 128, 32, q0, bh);
+          bulk_commit_group();
+        }
+      } else {
+        // d = 128: no shared memory is left for a separate staging buffer.  The dO tile of this
+        // block's stage is free once dV(it) has read it; it takes the scaled dQ block in two
+        // 64-column halves (two 32-column fp32 boxes each), bulk reduce-added one after the other.
+        // The 128 TMEM columns are read as four 32-column chunks, two loads in flight, and are
+        // released once the last chunk is in registers.
+        const int s = it % T::NS;
+        const uint32_t stg = sbase + T::OFF_QD + s * 2 * T::TILE_BYTES + T::TILE_BYTES;
+        auto stage = [&](const uint32_t (&v)[32], int box) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t addr = stg + box * (128 * 128) + r * 128 + ((c ^ (r & 7)) << 4);
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                         "f"(__uint_as_float(v[4 * c]) * p.scale), "f"(__uint_as_float(v[4 * c + 1]) * p.scale),
+                         "f"(__uint_as_float(v[4 * c + 2]) * p.scale), "f"(__uint_as_float(v[4 * c + 3]) * p.scale)
+                         : "memory");
+          }
+        };
+        auto reduce_half = [&](int h) {  // after the barrier that follows the half's staging
+          if (leader) {
+            // Rows past Nq fall outside the tensor map and are not written.
+            tma_reduce_add_3d(&tmDQ, stg, 64 * h, q0, bh);
+            tma_reduce_add_3d(&tmDQ, stg + 128 * 128, 64 * h + 32, q0, bh);
+            bulk_commit_group();
+            bulk_wait_group_read0();  // the staging buffer is read out
+          }
+          asm volatile("bar.sync 2, 128;" ::: "memory");
+        };
+        uint32_t va[32], vb[32];
+        if (ok) {
+          tc_fence_after();
+          tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DQ, va);
+          tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DQ + 32, vb);
+          tmem_wait_ld_2x32(va, vb);
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DO_FREE), it & 1, abort_flag));
+        }
+        if (ok) {
+          stage(va, 0);
+          stage(vb, 1);
+          tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DQ + 64, va);
+          tmem_ld32x32b_x32_nowait(lane_addr + T::COL_DQ + 96, vb);
+          tmem_wait_ld_2x32(va, vb);
+          tc_fence_before();
+          mbar_arrive(bar(T::BAR_DQ_FREE));
+          fence_proxy_async_smem();
+        }
+        if (!bar_sync_all(2, 128, ok)) {
+          ok = false;
+          break;
+        }
+        reduce_half(0);
+        stage(va, 0);
+        stage(vb, 1);
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 2, 128;" ::: "memory");
+        reduce_half(1);
+        if (leader && it + T::NS < n_q) mbar_arrive(bar(T::BAR_QD_EMPTY + s));
+      }
+    }
+    if (!ok) *abort_flag = 1;
+    if (leader) bulk_wait_group0();  // every reduce-add complete before the CTA exits
   } else if (warp == T::WARP_A || warp == T::WARP_B) {
     // ------------------------------------------------------------------ MMA issuers A and B
     // Each issuer is a whole converged warp (one elected lane issues), and each runs its own

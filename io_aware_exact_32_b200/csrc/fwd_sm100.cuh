@@ -567,7 +567,6 @@ __global__ void __launch_bounds__(FwdTraits<D, F8, EXT>::THREADS, 1)
       bool ok = true;
       int L = 0;                // global index of the item's first K/V load
       int cnt0 = 0, cnt1 = 0;   // S tiles of groups 0 / 1 in earlier items (barrier phases run on)
-      bool s0_early = false;    // this item's first S_0 was issued at the end of the previous item
       for (int k = 0; ok && item_at(k) < n_items; ++k) {
         const FwdItem w = decode(item_at(k));
         const int slot = k % T::QSLOTS;
@@ -626,7 +625,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8, EXT>::THREADS, 1)
             const int ik = L + 2 * j, iv = ik + 1;
             if (!(ok = kv_wait(ik))) break;
             tc_fence_after();
-            if (j < w.n0 && !(j == 0 && s0_early)) {
+            if (j < w.n0) {
               fwd_issue_qk<D, F8>(tS[0], q_smem[0], kv_smem(ik));
               mma_commit_w(bar(T::BAR_S_FULL + 0));
             }
@@ -644,29 +643,6 @@ __global__ void __launch_bounds__(FwdTraits<D, F8, EXT>::THREADS, 1)
               if (!(ok = pv(0, cnt0 + j, iv, j > 0))) break;
             }
             v_prev = iv;
-          }
-          // Group 0 is done with this item (tile 1 sees one more key tile).  The next item's first
-          // S_0 goes to the tensor pipe before the last P_1 V, which waits for group 1's last
-          // softmax, so that group 0 starts the next item meanwhile.  Its S buffer was last read by
-          // P_0 V of this item, its Q sits in the other slot (two slots only: with one, that slot
-          // is released after this item), and its first K tile only needs stages this item has
-          // already released.
-          s0_early = false;
-          if constexpr (T::QSLOTS == 2) {
-            if (ok && item_at(k + 1) < n_items) {
-              const FwdItem w1 = decode(item_at(k + 1));
-              const int slot1 = (k + 1) % T::QSLOTS;
-              if (w1.n0 > 0) {
-                ok = warp_wait(bar(T::BAR_Q_FULL + slot1), ((k + 1) / T::QSLOTS) & 1, abort_flag) &&
-                     kv_wait(L + 2 * w.n_kv);
-                if (ok) {
-                  tc_fence_after();
-                  fwd_issue_qk<D, F8>(tS[0], sbase + T::OFF_Q + (2 * slot1) * T::TILE_BYTES, kv_smem(L + 2 * w.n_kv));
-                  mma_commit_w(bar(T::BAR_S_FULL + 0));
-                  s0_early = true;
-                }
-              }
-            }
           }
           if (ok && w.n_kv == 1) ok = o_free(1);
           if (ok && (ok = pv(1, cnt1 + w.n_kv - 1, v_prev, w.n_kv - 1 > 0))) release(v_prev);
