@@ -273,26 +273,9 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     if constexpr (EXT) {
       if (p.bias != nullptr && key_ok) bias_col = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + key;
     }
-    // EXT: the bias entries (q, key) of one 16-column chunk of this group, as packed bf16 pairs
-    // (zero past Nq or without a bias).  Loaded one chunk ahead of their use (the first chunk
-    // before the block's waits), so that their latency stays off the P/dS chain.
-    auto load_bias = [&](int q0, int ch, uint32_t (&dst)[8]) {
-      const int qc = q0 + cb + 16 * ch;
-#pragma unroll
-      for (int e = 0; e < 16; e += 2) {
-        uint32_t lo = 0u, hi = 0u;
-        if (bias_col != nullptr && qc + e < p.Nq)
-          lo = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)(qc + e) * p.Nk));
-        if (bias_col != nullptr && qc + e + 1 < p.Nq)
-          hi = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)(qc + e + 1) * p.Nk));
-        dst[e / 2] = lo | (hi << 16);
-      }
-    };
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
       const int q0 = (i0 + it) * 128;
-      [[maybe_unused]] uint32_t braw[2][8];
-      if constexpr (EXT) load_bias(q0, 0, braw[0]);
       // Per-block statistics, stored negated: -LSE in log2 units (-inf past Nq) and -D.  The
       // first barrier keeps the previous block's readers ahead of the overwrite, the second
       // publishes the new values.
@@ -344,11 +327,20 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb + 16 * (ch + 1), dpv[cur ^ 1]);
         }
         uint32_t pk[8], dk[8];
-        // EXT: dropout decisions of this chunk's 16 query columns (bit e: column 16 ch + e kept).
+        // EXT: bias (log2 units, added to -LSE) and dropout decisions (bit e: column 16 ch + e kept)
+        // of this chunk's 16 query columns.
+        [[maybe_unused]] float badd[16];
         [[maybe_unused]] uint32_t keepm = 0xffffu;
         if constexpr (EXT) {
           const int qc = q0 + cb + 16 * ch;
-          if (ch < NCH - 1) load_bias(q0, ch + 1, braw[cur ^ 1]);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            badd[e] = 0.f;
+            if (bias_col != nullptr && qc + e < p.Nq) {
+              const unsigned short raw = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)(qc + e) * p.Nk));
+              badd[e] = __uint_as_float((uint32_t)raw << 16) * kLog2e;
+            }
+          }
           if (p.drop.p8 != 0) keepm = dropout_keep_colwise(p.drop, (uint32_t)(qc >> 2), (uint32_t)key, (uint32_t)bh, lane);
         }
 #pragma unroll
@@ -357,13 +349,10 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           float4 nl = st4[c >> 2];        // broadcast: every lane reads the same address
           const float4 nd = st4[32 + (c >> 2)];
           if constexpr (EXT) {
-            // bias (bf16 pairs) in log2 units, added to -LSE
-            const uint32_t b01 = braw[cur][i / 2], b23 = braw[cur][i / 2 + 1];
-            const float2 l01 = ffma2(make_float2(__uint_as_float(b01 << 16), __uint_as_float(b01 & 0xffff0000u)),
-                                     make_float2(kLog2e, kLog2e), make_float2(nl.x, nl.y));
-            const float2 l23 = ffma2(make_float2(__uint_as_float(b23 << 16), __uint_as_float(b23 & 0xffff0000u)),
-                                     make_float2(kLog2e, kLog2e), make_float2(nl.z, nl.w));
-            nl = make_float4(l01.x, l01.y, l23.x, l23.y);
+            nl.x += badd[i];
+            nl.y += badd[i + 1];
+            nl.z += badd[i + 2];
+            nl.w += badd[i + 3];
           }
           const float2 x01 = ffma2(make_float2(__uint_as_float(sv[cur][i]), __uint_as_float(sv[cur][i + 1])), sc2,
                                    make_float2(nl.x, nl.y));
