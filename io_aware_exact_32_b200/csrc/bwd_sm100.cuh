@@ -311,6 +311,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       const bool masked = __any_sync(0xffffffffu, !key_ok || cmin > cb);
       const float4* st4 = reinterpret_cast<const float4*>(stat);
       const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+      [[maybe_unused]] const float2 inv2 = make_float2(kLog2e / p.scale_log2, kLog2e / p.scale_log2);  // 1 / scale
       [[maybe_unused]] const float zscale = p.drop.p8 != 0 ? p.drop.scale : 1.f;
       // 16-column chunks, double-buffered: the load of chunk c+1 is issued right after chunk c
       // has arrived and overlaps its arithmetic (a TMEM load wait covers every load in flight).
@@ -327,8 +328,9 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb + 16 * (ch + 1), dpv[cur ^ 1]);
         }
         uint32_t pk[8], dk[8];
-        // EXT: bias (log2 units, added to -LSE) and dropout decisions (bit e: column 16 ch + e kept)
-        // of this chunk's 16 query columns.
+        // EXT: bias and dropout decisions (bit e: column 16 ch + e kept) of this chunk's 16 query
+        // columns.  The bias enters the unscaled score, s + bias / scale, so that the exponent's
+        // multiply-add by scale * log2(e) covers both.
         [[maybe_unused]] float badd[16];
         [[maybe_unused]] uint32_t keepm = 0xffffu;
         if constexpr (EXT) {
@@ -338,7 +340,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
             badd[e] = 0.f;
             if (bias_col != nullptr && qc + e < p.Nq) {
               const unsigned short raw = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)(qc + e) * p.Nk));
-              badd[e] = __uint_as_float((uint32_t)raw << 16) * kLog2e;
+              badd[e] = __uint_as_float((uint32_t)raw << 16);
             }
           }
           if (p.drop.p8 != 0) keepm = dropout_keep_colwise(p.drop, (uint32_t)(qc >> 2), (uint32_t)key, (uint32_t)bh, lane);
@@ -346,18 +348,16 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; i += 4) {
           const int c = cb + 16 * ch + i;
-          float4 nl = st4[c >> 2];        // broadcast: every lane reads the same address
+          const float4 nl = st4[c >> 2];  // broadcast: every lane reads the same address
           const float4 nd = st4[32 + (c >> 2)];
+          float2 s01 = make_float2(__uint_as_float(sv[cur][i]), __uint_as_float(sv[cur][i + 1]));
+          float2 s23 = make_float2(__uint_as_float(sv[cur][i + 2]), __uint_as_float(sv[cur][i + 3]));
           if constexpr (EXT) {
-            nl.x += badd[i];
-            nl.y += badd[i + 1];
-            nl.z += badd[i + 2];
-            nl.w += badd[i + 3];
+            s01 = ffma2(make_float2(badd[i], badd[i + 1]), inv2, s01);
+            s23 = ffma2(make_float2(badd[i + 2], badd[i + 3]), inv2, s23);
           }
-          const float2 x01 = ffma2(make_float2(__uint_as_float(sv[cur][i]), __uint_as_float(sv[cur][i + 1])), sc2,
-                                   make_float2(nl.x, nl.y));
-          const float2 x23 = ffma2(make_float2(__uint_as_float(sv[cur][i + 2]), __uint_as_float(sv[cur][i + 3])),
-                                   sc2, make_float2(nl.z, nl.w));
+          const float2 x01 = ffma2(s01, sc2, make_float2(nl.x, nl.y));
+          const float2 x23 = ffma2(s23, sc2, make_float2(nl.z, nl.w));
           float2 p01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
           float2 p23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
           if (masked) {

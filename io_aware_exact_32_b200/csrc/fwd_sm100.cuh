@@ -188,19 +188,24 @@ __device__ __forceinline__ float max64(const float* s) {
 }
 
 // Bias step of the EXT forward for the 64 keys of one row held in a staged bias box:
-// s <- s * scale_log2 + bias * log2(e).  The box is 128 rows of 128 bytes with 16-byte chunk c of row
-// r at ((c ^ (r % 8)) * 16) (the 128-byte swizzle of the TMA box); keys past Nk and rows past Nq
-// were filled with zeros by the TMA (those scores are -inf or never stored).
-__device__ __forceinline__ void fwd_apply_bias_smem(float* s, const uint8_t* box, int r, float scale_log2) {
-  constexpr float kLog2eF = 1.4426950408889634f;
+// s <- s + bias / scale (in pairs, one fused multiply-add each): the scores stay unscaled, as without
+// a bias, and scale * log2(e) enters with the row maximum in the exponent's multiply-add, so that
+// exp2((s + bias / scale) * scale * log2(e) - m) = exp(scale * s + bias) / 2^m.  The box is 128 rows of
+// 128 bytes with 16-byte chunk c of row r at ((c ^ (r % 8)) * 16) (the 128-byte swizzle of the TMA
+// box); keys past Nk and rows past Nq were filled with zeros by the TMA (those scores are -inf or
+// never stored).
+__device__ __forceinline__ void fwd_apply_bias_smem(float* s, const uint8_t* box, int r, float inv_scale) {
+  const float2 inv2 = make_float2(inv_scale, inv_scale);
 #pragma unroll
   for (int g = 0; g < 8; ++g) {
     const uint4 raw = *reinterpret_cast<const uint4*>(box + r * 128 + ((g ^ (r & 7)) << 4));
     const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      s[8 * g + 2 * i] = fmaf(s[8 * g + 2 * i], scale_log2, bf16lo_to_f32(w[i]) * kLog2eF);
-      s[8 * g + 2 * i + 1] = fmaf(s[8 * g + 2 * i + 1], scale_log2, bf16hi_to_f32(w[i]) * kLog2eF);
+      const float2 v = ffma2(make_float2(bf16lo_to_f32(w[i]), bf16hi_to_f32(w[i])), inv2,
+                             make_float2(s[8 * g + 2 * i], s[8 * g + 2 * i + 1]));
+      s[8 * g + 2 * i] = v.x;
+      s[8 * g + 2 * i + 1] = v.y;
     }
   }
 }
@@ -318,7 +323,8 @@ __global__ void __launch_bounds__(FwdTraits<D, F8, EXT>::THREADS, 1)
       if constexpr (F8) scale_log2 *= __ldg(p.descale_q + bh) * __ldg(p.descale_k + bh);
       // EXT: the scores are turned into log2-domain logits s * scale * log2(e) + bias * log2(e) in
       // place, so the exponent step below multiplies by 1.
-      const float2 sc2 = EXT ? make_float2(1.f, 1.f) : make_float2(scale_log2, scale_log2);
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      [[maybe_unused]] const float inv_scale = 1.4426950408889634f / scale_log2;  // EXT: 1 / scale
       // EXT with a bias: this group's staged bias tile, one 64-key box per half of the scores.
       const uint8_t* bias_box = smem + T::OFF_BIAS + t * T::BIAS_TILE;
       for (int step = 0; step < n_own; ++step) {
@@ -344,10 +350,7 @@ __global__ void __launch_bounds__(FwdTraits<D, F8, EXT>::THREADS, 1)
           if (staged_bias) {
             ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_BIAS_FULL + t), bcnt & 1, abort_flag));
             if (!ok) break;
-            fwd_apply_bias_smem(s, bias_box, r, scale_log2);
-          } else {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) s[c] *= scale_log2;
+            fwd_apply_bias_smem(s, bias_box, r, inv_scale);
           }
         }
         const float mx_a = max64(s);
@@ -359,16 +362,13 @@ __global__ void __launch_bounds__(FwdTraits<D, F8, EXT>::THREADS, 1)
         }
         if constexpr (EXT) {
           if (staged_bias) {
-            fwd_apply_bias_smem(s2, bias_box + T::BIAS_TILE / 2, r, scale_log2);
+            fwd_apply_bias_smem(s2, bias_box + T::BIAS_TILE / 2, r, inv_scale);
             mbar_arrive(bar(T::BAR_BIAS_EMPTY + t));  // this tile's bias has been read
             ++bcnt;
-          } else {
-#pragma unroll
-            for (int c = 0; c < 64; ++c) s2[c] *= scale_log2;
           }
         }
         const float mx = fmaxf(mx_a, max64(s2));
-        const float m_tile = EXT ? mx : mx * scale_log2;
+        const float m_tile = mx * scale_log2;
         float alpha = 1.f;
         bool resc = false;
         if (m_tile > m_run + kRescaleThreshold) {
