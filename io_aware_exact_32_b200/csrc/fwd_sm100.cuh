@@ -509,20 +509,8 @@ __global__ void __launch_bounds__(FwdTraits<D, F8, EXT>::THREADS, 1)
         const float inv = lr_run > 0.f ? num / lr_run : 0.f;
         const bool in_range = row < p.Nq;
         __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (in_range ? row : 0)) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32x32b_x32_wait(lane_addr + colO + 32 * c, o);
-          if (use1) {
-            uint32_t o1[32];
-            tmem_ld32x32b_x32_wait(lane_addr + T::col_o(1) + 32 * c, o1);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              o[i] = __float_as_uint(a0 * __uint_as_float(o[i]) + a1 * __uint_as_float(o1[i]));
-          } else if (!two) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(a0 * __uint_as_float(o[i]));
-          }
+        // O chunk c (32 columns, already combined) / l -> bf16 -> the output row.
+        auto put = [&](const uint32_t (&o)[32], int c) {
           uint32_t wv[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -532,10 +520,51 @@ __global__ void __launch_bounds__(FwdTraits<D, F8, EXT>::THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
           }
+        };
+        bool released = false;  // O_FREE already signalled
+        if constexpr (F8) {
+          if (two) {
+            // FP8, two-tile mode (measured faster there, not with bf16 operands): the four 32-column
+            // chunks of O_t with loads in flight while earlier chunks are stored (a TMEM load wait
+            // covers every load in flight), and the columns released as soon as the last chunk is in
+            // registers.
+            uint32_t oa[32], ob[32], oc[32];
+            tmem_ld32x32b_x32_nowait(lane_addr + colO, oa);
+            tmem_ld32x32b_x32_nowait(lane_addr + colO + 32, ob);
+            tmem_wait_ld_2x32(oa, ob);
+            tmem_ld32x32b_x32_nowait(lane_addr + colO + 64, oc);
+            put(oa, 0);
+            tmem_ld32x32b_x32_nowait(lane_addr + colO + 96, oa);
+            put(ob, 1);
+            tmem_wait_ld_2x32(oc, oa);
+            tc_fence_before();
+            mbar_arrive(bar(T::BAR_O_FREE + t));
+            released = true;
+            put(oc, 2);
+            put(oa, 3);
+          }
         }
-        // O_t is in registers and on its way out: the next item's first P V may overwrite it.
-        tc_fence_before();
-        mbar_arrive(bar(T::BAR_O_FREE + t));
+        if (!released) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32x32b_x32_wait(lane_addr + colO + 32 * c, o);
+            if (use1) {
+              uint32_t o1[32];
+              tmem_ld32x32b_x32_wait(lane_addr + T::col_o(1) + 32 * c, o1);
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                o[i] = __float_as_uint(a0 * __uint_as_float(o[i]) + a1 * __uint_as_float(o1[i]));
+            } else if (!two) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(a0 * __uint_as_float(o[i]));
+            }
+            put(o, c);
+          }
+          // O_t is in registers and on its way out: the next item's first P V may overwrite it.
+          tc_fence_before();
+          mbar_arrive(bar(T::BAR_O_FREE + t));
+        }
         if (in_range) p.lse[(size_t)bh * p.Nq + row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
       }
     }
