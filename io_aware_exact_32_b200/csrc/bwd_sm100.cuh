@@ -268,10 +268,12 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     // Query column c of block i sees this key iff c >= cmin (bottom-right causal alignment).
     const int shift = key - (p.Nk - p.Nq);
     const uint32_t ds_row = sbase + T::OFF_DS + r * 128;
-    // EXT: this key's column of the bias (element (q, key) at bias_col[q * Nk]).
+    // EXT: this key's column of the bias (element (q, key) at bias_col[q * Nk]).  A key past Nk reads
+    // key 0's column instead (its weights are masked to 0), so the loads need no per-thread guard.
+    [[maybe_unused]] const bool has_bias = EXT && p.bias != nullptr;  // uniform over the CTA
     const __nv_bfloat16* bias_col = nullptr;
     if constexpr (EXT) {
-      if (p.bias != nullptr && key_ok) bias_col = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + key;
+      if (has_bias) bias_col = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + (key_ok ? key : 0);
     }
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
@@ -335,11 +337,13 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
         [[maybe_unused]] uint32_t keepm = 0xffffu;
         if constexpr (EXT) {
           const int qc = q0 + cb + 16 * ch;
+          if (has_bias) {
+            // A query row past Nq reads row Nq - 1 instead: its LSE is -inf, so its weight is 0 whatever
+            // the bias (never +inf, so no NaN).
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            badd[e] = 0.f;
-            if (bias_col != nullptr && qc + e < p.Nq) {
-              const unsigned short raw = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)(qc + e) * p.Nk));
+            for (int e = 0; e < 16; ++e) {
+              const int q = min(qc + e, p.Nq - 1);
+              const unsigned short raw = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)q * p.Nk));
               badd[e] = __uint_as_float((uint32_t)raw << 16);
             }
           }
@@ -353,8 +357,10 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           float2 s01 = make_float2(__uint_as_float(sv[cur][i]), __uint_as_float(sv[cur][i + 1]));
           float2 s23 = make_float2(__uint_as_float(sv[cur][i + 2]), __uint_as_float(sv[cur][i + 3]));
           if constexpr (EXT) {
-            s01 = ffma2(make_float2(badd[i], badd[i + 1]), inv2, s01);
-            s23 = ffma2(make_float2(badd[i + 2], badd[i + 3]), inv2, s23);
+            if (has_bias) {
+              s01 = ffma2(make_float2(badd[i], badd[i + 1]), inv2, s01);
+              s23 = ffma2(make_float2(badd[i + 2], badd[i + 3]), inv2, s23);
+            }
           }
           const float2 x01 = ffma2(s01, sc2, make_float2(nl.x, nl.y));
           const float2 x23 = ffma2(s23, sc2, make_float2(nl.z, nl.w));

@@ -5,11 +5,11 @@ records FA_ERR_TIMEOUT in the device status word, the other warps of the CTA
 see its abort flag and stop, and the teardown still waits (with the fixed 2 s
 limit) for the CTA's own copies and MMAs in flight before it frees its tensor
 memory and exits.  Here the test hook fa_debug_set_wait_limit lowers the
-limit to 300 ns, so the waits of a healthy causal forward (or backward) run
-out; the test checks that fa_get_device_error reports the timeout, restores
-the limit, and checks that the next call on the same device matches the
-float64 oracle (nothing was left allocated or half-written that it could trip
-over).
+limit to 300 ns, so the waits of a healthy causal forward, backward (both
+head dims) or split-KV decode run out; each test checks that
+fa_get_device_error reports the timeout, restores the limit, and checks that
+the next call on the same device matches the float64 oracle (nothing was left
+allocated or half-written that it could trip over).
 """
 import math
 
@@ -58,8 +58,10 @@ def test_waits_give_up_and_the_device_stays_usable():
     assert np.isfinite(gc.f64(o2)).all()
 
 
-def test_backward_waits_give_up_and_the_device_stays_usable():
-    B, H, N, d = 1, 16, 4096, 128
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_waits_give_up_and_the_device_stays_usable(d):
+    # d = 64 and d = 128 take different dQ paths (own staging buffer / the block's dO tile).
+    B, H, N = 1, 16, 4096
     x = W.make_attention_inputs(B, H, N, N, d, seed=92, with_do=True)
     q, k, v, do = gc.to_dev(x["q"], x["k"], x["v"], x["do"])
     scale = 1.0 / math.sqrt(d)
@@ -85,3 +87,28 @@ def test_backward_waits_give_up_and_the_device_stays_usable():
     check_grad(gc.f64(dq[0, h]), rdq, "dQ")
     check_grad(gc.f64(dk[0, h]), rdk, "dK")
     check_grad(gc.f64(dv[0, h]), rdv, "dV")
+
+
+def test_decode_waits_give_up_and_the_device_stays_usable():
+    x = W.make_decode_inputs(8, 8, 4096, 128, 1024, seed=93)
+    q, kc, vc = gc.to_dev(x["q"], x["k_cache"], x["v_cache"])
+    seq = x["seqlens"].to(gc.DEV)
+    scale = 1.0 / math.sqrt(128)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    fa.fa_debug_set_wait_limit(300)
+    try:
+        fa.decode_splitkv(q, kc, vc, seq, scale=scale)
+        torch.cuda.synchronize()
+        status = fa.fa_get_device_error()
+    finally:
+        fa.fa_debug_set_wait_limit(0)
+    assert status == FA_ERR_TIMEOUT, status
+
+    o, lse = fa.decode_splitkv(q, kc, vc, seq, scale=scale)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_error() == 0
+    o_ref, l_ref = A.decode_forward(gc.f64(x["q"]), gc.f64(x["k_cache"]), gc.f64(x["v_cache"]),
+                                    x["seqlens"].numpy(), scale)
+    check_o(gc.f64(o)[:, :, 0], o_ref)
+    check_lse(gc.f64(lse), l_ref)
