@@ -275,9 +275,27 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
     if constexpr (EXT) {
       if (has_bias) bias_col = p.bias + (bh / p.H) * p.bias_sb + (bh % p.H) * p.bias_sh + (key_ok ? key : 0);
     }
+    // EXT: the bias entries (q, key) of one 16-column chunk of this group as packed bf16 pairs, loaded
+    // one chunk ahead of their use (the first chunk before the block's waits) so that their latency
+    // stays off the P/dS chain.  A query row past Nq reads row Nq - 1 instead: its LSE is -inf, so its
+    // weight is 0 whatever the bias (never +inf, so no NaN).
+    auto load_bias = [&](int q0, int ch, uint32_t (&dst)[8]) {
+      const int qc = q0 + cb + 16 * ch;
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
+        const int qa = min(qc + e, p.Nq - 1), qb = min(qc + e + 1, p.Nq - 1);
+        const uint32_t lo = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)qa * p.Nk));
+        const uint32_t hi = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)qb * p.Nk));
+        dst[e / 2] = lo | (hi << 16);
+      }
+    };
     bool ok = true;
     for (int it = 0; it < n_q; ++it) {
       const int q0 = (i0 + it) * 128;
+      [[maybe_unused]] uint32_t braw[2][8];
+      if constexpr (EXT) {
+        if (has_bias) load_bias(q0, 0, braw[0]);
+      }
       // Per-block statistics, stored negated: -LSE in log2 units (-inf past Nq) and -D.  The
       // first barrier keeps the previous block's readers ahead of the overwrite, the second
       // publishes the new values.
@@ -333,20 +351,10 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
         // EXT: bias and dropout decisions (bit e: column 16 ch + e kept) of this chunk's 16 query
         // columns.  The bias enters the unscaled score, s + bias / scale, so that the exponent's
         // multiply-add by scale * log2(e) covers both.
-        [[maybe_unused]] float badd[16];
         [[maybe_unused]] uint32_t keepm = 0xffffu;
         if constexpr (EXT) {
           const int qc = q0 + cb + 16 * ch;
-          if (has_bias) {
-            // A query row past Nq reads row Nq - 1 instead: its LSE is -inf, so its weight is 0 whatever
-            // the bias (never +inf, so no NaN).
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int q = min(qc + e, p.Nq - 1);
-              const unsigned short raw = __ldg(reinterpret_cast<const unsigned short*>(bias_col + (size_t)q * p.Nk));
-              badd[e] = __uint_as_float((uint32_t)raw << 16);
-            }
-          }
+          if (has_bias && ch < NCH - 1) load_bias(q0, ch + 1, braw[cur ^ 1]);
           if (p.drop.p8 != 0) keepm = dropout_keep_colwise(p.drop, (uint32_t)(qc >> 2), (uint32_t)key, (uint32_t)bh, lane);
         }
 #pragma unroll
@@ -358,8 +366,9 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
           float2 s23 = make_float2(__uint_as_float(sv[cur][i + 2]), __uint_as_float(sv[cur][i + 3]));
           if constexpr (EXT) {
             if (has_bias) {
-              s01 = ffma2(make_float2(badd[i], badd[i + 1]), inv2, s01);
-              s23 = ffma2(make_float2(badd[i + 2], badd[i + 3]), inv2, s23);
+              const uint32_t b01 = braw[cur][i / 2], b23 = braw[cur][i / 2 + 1];
+              s01 = ffma2(make_float2(__uint_as_float(b01 << 16), __uint_as_float(b01 & 0xffff0000u)), inv2, s01);
+              s23 = ffma2(make_float2(__uint_as_float(b23 << 16), __uint_as_float(b23 & 0xffff0000u)), inv2, s23);
             }
           }
           const float2 x01 = ffma2(s01, sc2, make_float2(nl.x, nl.y));
