@@ -30,10 +30,8 @@
 // Two issuers because one thread issues at most one 128 x N x 16 MMA every ~115 cycles
 // (measured on B200), about half the tensor-core rate at N = 128.  Each issuer runs one
 // iteration ahead: right after the MMAs that consume block i it issues the next block's S^T /
-// dP^T, so the compute warps wait only for those.  S^T and dP^T have a barrier each, so that the
-// P/dS threads start a block's weights on S^T while its dP^T, which the tensor pipe finishes after
-// S^T, is still being computed.  Barriers that must see both issuers' work (a Q/dO stage free,
-// final dK/dV) count two commits.
+// dP^T, so the compute warps wait only for those.  Barriers that must see both issuers' work
+// (S^T and dP^T ready, a Q/dO stage free, final dK/dV) count two commits.
 #pragma once
 
 #include <type_traits>
@@ -77,8 +75,7 @@ struct BwdTraits {
   static constexpr int BAR_P_FREE = BAR_S_FULL + 9;   // dV(i) has read P^T(i)
   static constexpr int BAR_DO_FREE = BAR_S_FULL + 10; // dV(i) has read dO(i) (d = 128: staging)
   static constexpr int BAR_DQ_ISSUED = BAR_S_FULL + 11;  // issuer B has issued dQ(i): issuer A may issue dV(i)
-  static constexpr int BAR_DP_FULL = BAR_S_FULL + 12;    // dP^T(i) complete (S_FULL: S^T(i) complete)
-  static constexpr int NBAR = BAR_DP_FULL + 1;
+  static constexpr int NBAR = BAR_DQ_ISSUED + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -228,8 +225,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       // dO tile is read out (d = 128)
       mbar_init(bar(T::BAR_QD_EMPTY + s), 2);
     }
-    mbar_init(bar(T::BAR_S_FULL), 1);   // issuer A after S^T
-    mbar_init(bar(T::BAR_DP_FULL), 1);  // issuer B after dP^T
+    mbar_init(bar(T::BAR_S_FULL), 2);  // issuer A after S^T, issuer B after dP^T
     mbar_init(bar(T::BAR_DS_READY), 128 * T::NCWG);
     mbar_init(bar(T::BAR_DS_FREE), 1);  // issuer B after dQ and dK (the readers of dS^T)
     mbar_init(bar(T::BAR_DQ_FULL), 1);
@@ -342,32 +338,30 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       constexpr int NCH = T::CW / 16;  // 16-column chunks of this group
       uint32_t sv[2][16], dpv[2][16];
       tmem_ld32x32b_x16_nowait(lane_addr + T::COL_S + cb, sv[0]);
-      tmem_wait_ld_x16(sv[0]);
+      tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb, dpv[0]);
+      tmem_wait_ld_2x16(sv[0], dpv[0]);
 #pragma unroll
       for (int ch = 0; ch < NCH; ++ch) {
         const int cur = ch & 1;
-        if (ch > 0 && ch < NCH - 1) {
+        if (ch < NCH - 1) {
           tmem_ld32x32b_x16_nowait(lane_addr + T::COL_S + cb + 16 * (ch + 1), sv[cur ^ 1]);
           tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb + 16 * (ch + 1), dpv[cur ^ 1]);
         }
         uint32_t pk[8], dk[8];
-        // EXT: dropout decisions (bit e: column 16 ch + e kept) of this chunk's 16 query columns.  The
-        // bias enters the unscaled score, s + bias / scale, so that the exponent's multiply-add by
-        // scale * log2(e) covers both.
+        // EXT: bias and dropout decisions (bit e: column 16 ch + e kept) of this chunk's 16 query
+        // columns.  The bias enters the unscaled score, s + bias / scale, so that the exponent's
+        // multiply-add by scale * log2(e) covers both.
         [[maybe_unused]] uint32_t keepm = 0xffffu;
         if constexpr (EXT) {
           const int qc = q0 + cb + 16 * ch;
           if (has_bias && ch < NCH - 1) load_bias(q0, ch + 1, braw[cur ^ 1]);
           if (p.drop.p8 != 0) keepm = dropout_keep_colwise(p.drop, (uint32_t)(qc >> 2), (uint32_t)key, (uint32_t)bh, lane);
         }
-        // Phase 1, from S^T alone: the weights of the chunk's 16 columns and their P^T (dropped and
-        // rescaled with EXT).
-        float2 pw[8];
-        [[maybe_unused]] float2 zw[8];  // EXT: dropout factors (kept: 1 / (1 - p), dropped: 0)
 #pragma unroll
         for (int i = 0; i < 16; i += 4) {
           const int c = cb + 16 * ch + i;
           const float4 nl = st4[c >> 2];  // broadcast: every lane reads the same address
+          const float4 nd = st4[32 + (c >> 2)];
           float2 s01 = make_float2(__uint_as_float(sv[cur][i]), __uint_as_float(sv[cur][i + 1]));
           float2 s23 = make_float2(__uint_as_float(sv[cur][i + 2]), __uint_as_float(sv[cur][i + 3]));
           if constexpr (EXT) {
@@ -387,14 +381,23 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
             p23.x = (key_ok && c + 2 >= cmin) ? p23.x : 0.f;
             p23.y = (key_ok && c + 3 >= cmin) ? p23.y : 0.f;
           }
-          pw[i / 2] = p01;
-          pw[i / 2 + 1] = p23;
+          float2 t01, t23;
+          [[maybe_unused]] float2 z01, z23;  // EXT: dropout factors (kept: 1 / (1 - p), dropped: 0)
           if constexpr (EXT) {
-            const float2 z01 = make_float2(((keepm >> i) & 1u) ? zscale : 0.f, ((keepm >> (i + 1)) & 1u) ? zscale : 0.f);
-            const float2 z23 =
-                make_float2(((keepm >> (i + 2)) & 1u) ? zscale : 0.f, ((keepm >> (i + 3)) & 1u) ? zscale : 0.f);
-            zw[i / 2] = z01;
-            zw[i / 2 + 1] = z23;
+            z01 = make_float2(((keepm >> i) & 1u) ? zscale : 0.f, ((keepm >> (i + 1)) & 1u) ? zscale : 0.f);
+            z23 = make_float2(((keepm >> (i + 2)) & 1u) ? zscale : 0.f, ((keepm >> (i + 3)) & 1u) ? zscale : 0.f);
+            t01 = ffma2(make_float2(__uint_as_float(dpv[cur][i]), __uint_as_float(dpv[cur][i + 1])), z01,
+                        make_float2(nd.x, nd.y));
+            t23 = ffma2(make_float2(__uint_as_float(dpv[cur][i + 2]), __uint_as_float(dpv[cur][i + 3])), z23,
+                        make_float2(nd.z, nd.w));
+          } else {
+            t01 = fadd2(make_float2(__uint_as_float(dpv[cur][i]), __uint_as_float(dpv[cur][i + 1])),
+                        make_float2(nd.x, nd.y));
+            t23 = fadd2(make_float2(__uint_as_float(dpv[cur][i + 2]), __uint_as_float(dpv[cur][i + 3])),
+                        make_float2(nd.z, nd.w));
+          }
+          const float2 d01 = fmul2(p01, t01), d23 = fmul2(p23, t23);
+          if constexpr (EXT) {
             const float2 pz01 = fmul2(p01, z01);
             const float2 pz23 = fmul2(p23, z23);
             pk[i / 2] = pack_bf16x2(pz01.x, pz01.y);
@@ -403,37 +406,6 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
             pk[i / 2] = pack_bf16x2(p01.x, p01.y);
             pk[i / 2 + 1] = pack_bf16x2(p23.x, p23.y);
           }
-        }
-        if (ch == 0) {
-          // dP^T of this block: the tensor pipe completes it after S^T, and the weights above were
-          // computed meanwhile.  Then the next chunk's loads go out.
-          if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(T::BAR_DP_FULL), it & 1, abort_flag));
-          tc_fence_after();
-          tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb, dpv[0]);
-          tmem_wait_ld_x16(dpv[0]);
-          if (NCH > 1) {
-            tmem_ld32x32b_x16_nowait(lane_addr + T::COL_S + cb + 16, sv[1]);
-            tmem_ld32x32b_x16_nowait(lane_addr + T::COL_DP + cb + 16, dpv[1]);
-          }
-        }
-        // Phase 2: dS = P o (dP o Z - D).
-#pragma unroll
-        for (int i = 0; i < 16; i += 4) {
-          const int c = cb + 16 * ch + i;
-          const float4 nd = st4[32 + (c >> 2)];
-          float2 t01, t23;
-          if constexpr (EXT) {
-            t01 = ffma2(make_float2(__uint_as_float(dpv[cur][i]), __uint_as_float(dpv[cur][i + 1])), zw[i / 2],
-                        make_float2(nd.x, nd.y));
-            t23 = ffma2(make_float2(__uint_as_float(dpv[cur][i + 2]), __uint_as_float(dpv[cur][i + 3])), zw[i / 2 + 1],
-                        make_float2(nd.z, nd.w));
-          } else {
-            t01 = fadd2(make_float2(__uint_as_float(dpv[cur][i]), __uint_as_float(dpv[cur][i + 1])),
-                        make_float2(nd.x, nd.y));
-            t23 = fadd2(make_float2(__uint_as_float(dpv[cur][i + 2]), __uint_as_float(dpv[cur][i + 3])),
-                        make_float2(nd.z, nd.w));
-          }
-          const float2 d01 = fmul2(pw[i / 2], t01), d23 = fmul2(pw[i / 2 + 1], t23);
           dk[i / 2] = pack_bf16x2(d01.x, d01.y);
           dk[i / 2 + 1] = pack_bf16x2(d23.x, d23.y);
         }
@@ -632,7 +604,7 @@ __global__ void __launch_bounds__(BwdTraits<D>::THREADS, 1)
       auto issue_first = [&](int it) {
         if constexpr (is_a) bwd_issue_ss_kmajor<D>(tS, k_smem, q_smem(it));
         else bwd_issue_ss_kmajor<D>(tDP, v_smem, q_smem(it) + T::TILE_BYTES);
-        mma_commit_w(bar(is_a ? T::BAR_S_FULL : T::BAR_DP_FULL));
+        mma_commit_w(bar(T::BAR_S_FULL));
       };
       const uint64_t ds_kmaj = make_sdesc_sw128(ds_smem, 16, 1024);           // dS^T as A, K-major
       const uint64_t ds_mn = make_sdesc_sw128(ds_smem, T::BOX_BYTES, 1024);    // dS as A, MN-major
